@@ -1,0 +1,147 @@
+// capi.cu -- the compute entry points of the C ABI: argument checks on the
+// host, then the plan kernel and the delta kernels on the caller's stream.
+// No call here allocates memory or synchronises the host.
+#include <algorithm>
+
+#include "internal.cuh"
+
+using namespace lora;
+
+namespace {
+
+int check_call(const lora_pool *p, int target, int T, const void *ws, size_t ws_bytes) {
+  if (!p) return LORA_ERR_INVALID_ARG;
+  if (target < 0 || target >= p->n_targets) return LORA_ERR_INVALID_ARG;
+  if (T < 0 || T > kMaxTokens) return LORA_ERR_INVALID_ARG;
+  if (T == 0) return LORA_OK;
+  if (!ws) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return LORA_ERR_ALIGNMENT;
+  if (ws_bytes < plan_layout(T).total) return LORA_ERR_WORKSPACE;
+  return LORA_OK;
+}
+
+int check_rows(const void *ptr, int ld, int width) {
+  if (!ptr) return LORA_ERR_INVALID_ARG;
+  if (ld < width) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(ptr) || (ld % 8) != 0) return LORA_ERR_ALIGNMENT;
+  return LORA_OK;
+}
+
+// x and y must not overlap (x is read while y is written).
+bool overlap(const void *x, int ldx, const void *y, int ldy, int T) {
+  const char *xa = static_cast<const char *>(x), *ya = static_cast<const char *>(y);
+  const char *xb = xa + size_t(T) * ldx * 2, *yb = ya + size_t(T) * ldy * 2;
+  return xa < yb && ya < xb;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lora_workspace_bytes(const lora_pool *p, int target, int max_tokens) {
+  if (!p || target < 0 || target >= p->n_targets || max_tokens < 0 || max_tokens > kMaxTokens) return 0;
+  return plan_layout(max_tokens).total;
+}
+
+int lora_plan_layout_get(const lora_pool *p, int T, lora_plan_layout *out) {
+  if (!p || !out || T < 0 || T > kMaxTokens) return LORA_ERR_INVALID_ARG;
+  PlanLayout L = plan_layout(T);
+  out->header = L.header;
+  out->perm = L.perm;
+  out->seg_start = L.seg_start;
+  out->seg_slot = L.seg_slot;
+  out->items = L.items;
+  out->tiles = L.tiles;
+  out->total = L.total;
+  out->s_max = L.s_max;
+  out->i_max = L.i_max;
+  out->j_max = L.j_max;
+  return LORA_OK;
+}
+
+int lora_mma_min_rows(void) { return kMmaMinRows; }
+
+int lora_plan_ids(lora_pool *p, const int32_t *ids, int T, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_call(p, 0, T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  if (!ids) return LORA_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  return launch_plan_ids(p, ids, T, ws, static_cast<cudaStream_t>(stream));
+}
+
+int lora_plan_segments(lora_pool *p, const int32_t *seg_offsets, const int32_t *seg_slot, int S, int T, void *ws,
+                       size_t ws_bytes, void *stream) {
+  int rc = check_call(p, 0, T, ws, ws_bytes);
+  if (rc != LORA_OK) return rc;
+  if (S < 0 || S > kMaxTokens) return LORA_ERR_INVALID_ARG;
+  if (T == 0) return LORA_OK;
+  if (S > 0 && (!seg_offsets || !seg_slot)) return LORA_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  return launch_plan_segments(p, seg_offsets, seg_slot, S, T, ws, static_cast<cudaStream_t>(stream));
+}
+
+int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const float *scales, int T,
+                    const void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_call(p, target, T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
+  if (!scales) return LORA_ERR_INVALID_ARG;
+  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  return launch_decode(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const int32_t *ids,
+               const float *scales, int T, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_call(p, target, T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
+  if (!scales || !ids) return LORA_ERR_INVALID_ARG;
+  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
+  return lora_apply_plan(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, stream);
+}
+
+int lora_apply_segments(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
+                        const int32_t *seg_offsets, const int32_t *seg_slot, int S, const float *scales, int T,
+                        void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_call(p, target, T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
+  if (!scales) return LORA_ERR_INVALID_ARG;
+  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  if ((rc = lora_plan_segments(p, seg_offsets, seg_slot, S, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
+  return lora_apply_plan(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, stream);
+}
+
+int lora_shrink(lora_pool *p, int target, const void *x, int ldx, const int32_t *ids, int T, float *v, int ldv,
+                void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_call(p, target, T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
+  if (!ids || !v || ldv < p->r_max) return LORA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(v) & 3u) return LORA_ERR_ALIGNMENT;
+  if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
+  DeviceGuard g(p->device);
+  return launch_decode(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, ldv, T, ws,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int lora_expand(lora_pool *p, int target, const float *v, int ldv, void *y, int ldy, const int32_t *ids,
+                const float *scales, int T, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_call(p, target, T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
+  if (!ids || !v || !scales || ldv < p->r_max) return LORA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(v) & 3u) return LORA_ERR_ALIGNMENT;
+  if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
+  DeviceGuard g(p->device);
+  return launch_decode(p, kExpandOnly, target, nullptr, 0, y, ldy, scales, const_cast<float *>(v), ldv, T, ws,
+                       static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,271 @@
+// internal.cuh -- shared definitions of the B200 multi-LoRA delta library.
+//
+// Device-side views of the adapter pool and of a batch plan, the plan layout
+// inside the caller's workspace, and the handful of sm_100a PTX wrappers the
+// kernels use (mbarriers, 1-D bulk async copies, grid-dependency control,
+// bounded waits).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "lora.h"
+
+namespace lora {
+
+// ---------------------------------------------------------------- limits
+constexpr int kRMax = 64;            // largest slot rank
+constexpr int kMaxSlots = 16384;     // plan kernel keeps one counter per slot in smem
+constexpr int kMaxTargets = 4096;
+constexpr int kMaxTokens = 1 << 20;
+constexpr int kItemRows = 16;        // rows per decode work item
+constexpr int kTileVecs = 32;        // 16-byte vectors per pipeline tile row (512 B)
+constexpr int kTileRowBytes = kTileVecs * 16;
+constexpr int kMmaRows = 128;        // rows per tensor-core tile
+constexpr int kMmaMinRows = 1 << 30; // segment length that selects the tensor-core path
+constexpr int kPlanThreads = 1024;
+constexpr int kDecodeThreads = 256;
+constexpr int kClusterCtas = 8;      // CTAs that split one work item (portable cluster)
+constexpr int kStages = 4;           // pipeline depth of the decode kernel
+
+extern std::atomic<uint64_t> g_launches;
+
+// ---------------------------------------------------------------- views
+struct PoolView {
+  const uint8_t *base;     // page memory
+  const int32_t *pt;       // [n_slots][pps] physical page, -1 = none
+  const int32_t *rank;     // [n_slots][n_targets] rank of the adapter on a target
+  const int32_t *loaded;   // [n_slots] 1 = slot holds pages
+  long long page_bytes;
+  int pps;                 // pages per slot
+  int log2_page;           // -1: one page per slot
+  int n_slots;
+  int n_targets;
+};
+
+// Physical address of logical byte `off` of `slot`, and how many bytes stay
+// on the same page from there.
+__device__ __forceinline__ const uint8_t *pool_addr(const PoolView &p, int slot,
+                                                    long long off, long long *room) {
+  long long page_idx, inside;
+  if (p.log2_page < 0) {
+    page_idx = 0;
+    inside = off;
+    *room = p.page_bytes - off;
+  } else {
+    page_idx = off >> p.log2_page;
+    inside = off & (p.page_bytes - 1);
+    *room = p.page_bytes - inside;
+  }
+  int phys = __ldg(p.pt + (long long)slot * p.pps + page_idx);
+  if (phys < 0) return nullptr;
+  return p.base + (long long)phys * p.page_bytes + inside;
+}
+
+// Plan arrays inside the workspace (byte offsets from its base).
+struct PlanLayout {
+  size_t header, perm, seg_start, seg_slot, seg_row, items, tiles, total;
+  int s_max, i_max, j_max;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline PlanLayout plan_layout(int T) {
+  PlanLayout L;
+  int t = T > 0 ? T : 1;
+  L.s_max = t;
+  L.i_max = t + (t + kItemRows - 1) / kItemRows;
+  L.j_max = (3 * t + kMmaRows - 1) / kMmaRows + 1;
+  size_t off = 0;
+  L.header = off;    off = align256(off + 64 * 4);
+  L.perm = off;      off = align256(off + size_t(t) * 4);
+  L.seg_start = off; off = align256(off + size_t(L.s_max + 1) * 4);
+  L.seg_slot = off;  off = align256(off + size_t(L.s_max) * 4);
+  L.seg_row = off;   off = align256(off + size_t(L.s_max) * 4);
+  L.items = off;     off = align256(off + size_t(L.i_max) * 16);
+  L.tiles = off;     off = align256(off + size_t(L.j_max) * 16);
+  L.total = off;
+  return L;
+}
+
+// Header words of a plan.
+enum { kHdrSegs = 0, kHdrActive = 1, kHdrItems = 2, kHdrTiles = 3, kHdrT = 4 };
+
+struct PlanView {
+  int32_t *hdr;
+  int32_t *perm;
+  int32_t *seg_start;
+  int32_t *seg_slot;
+  int32_t *seg_row;
+  int4 *items;   // {slot, first perm index, rows, segment}
+  int4 *tiles;   // {slot, first row, rows, segment}
+};
+
+inline PlanView plan_view(void *ws, const PlanLayout &L) {
+  uint8_t *b = static_cast<uint8_t *>(ws);
+  PlanView v;
+  v.hdr = reinterpret_cast<int32_t *>(b + L.header);
+  v.perm = reinterpret_cast<int32_t *>(b + L.perm);
+  v.seg_start = reinterpret_cast<int32_t *>(b + L.seg_start);
+  v.seg_slot = reinterpret_cast<int32_t *>(b + L.seg_slot);
+  v.seg_row = reinterpret_cast<int32_t *>(b + L.seg_row);
+  v.items = reinterpret_cast<int4 *>(b + L.items);
+  v.tiles = reinterpret_cast<int4 *>(b + L.tiles);
+  return v;
+}
+
+// ---------------------------------------------------------------- PTX
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make mbarrier initialisation visible to the async (bulk copy) proxy.
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for an mbarrier phase with an iteration cap and a 1 s wall-clock cap.
+// On giving up, records LORA_ERR_TIMEOUT in the sticky status and returns
+// false; the caller skips the work that needed the data.
+constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr uint64_t kSpinNs = 1000000000ull;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u && global_timer_ns() - t0 > kSpinNs) break;
+  }
+  atomicCAS(status, 0, LORA_ERR_TIMEOUT);
+  return false;
+}
+
+// 1-D bulk async copy global -> this CTA's shared memory, completing on an
+// mbarrier (no multicast).  dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Programmatic dependent launch: wait for the grids this one depends on.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// bf16 pair <-> fp32 (exact decode; round-to-nearest-even encode).
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+__device__ __forceinline__ void unpack8(const uint4 &u, float f[8]) {
+  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x);
+  f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z);
+  f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void set_status(int *status, int code) { atomicCAS(status, 0, code); }
+
+}  // namespace lora
+
+// ---------------------------------------------------------------- host pool
+struct lora_pool {
+  int device = 0;
+  int n_targets = 0, r_max = 0, n_slots = 0;
+  std::vector<lora_target> targets;
+  std::vector<long long> a_off, bt_off;
+  long long slot_bytes = 0;
+  long long page_bytes = 0;
+  int pps = 0, log2_page = -1;
+  int n_pages = 0;
+  uint8_t *mem = nullptr;
+  size_t mem_bytes = 0;
+  std::vector<int32_t> free_pages;  // stack; back() is handed out next
+  std::vector<int32_t> pt, rank, loaded;
+  void *dev_tables = nullptr;
+  int32_t *d_pt = nullptr, *d_rank = nullptr, *d_loaded = nullptr;
+  int *d_status = nullptr;
+  int decode_smem = 0;
+  int decode_max_clusters = 0;
+  std::mutex mu;
+
+  lora::PoolView view() const {
+    lora::PoolView v;
+    v.base = mem;
+    v.pt = d_pt;
+    v.rank = d_rank;
+    v.loaded = d_loaded;
+    v.page_bytes = page_bytes;
+    v.pps = pps;
+    v.log2_page = log2_page;
+    v.n_slots = n_slots;
+    v.n_targets = n_targets;
+    return v;
+  }
+};
+
+namespace lora {
+
+// Makes the pool's device current for the scope of a call.
+struct DeviceGuard {
+  int prev = -1, want = -1;
+  explicit DeviceGuard(int d) : want(d) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != d) cudaSetDevice(d);
+  }
+  ~DeviceGuard() {
+    if (prev >= 0 && prev != want) cudaSetDevice(prev);
+  }
+};
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launchers (defined in plan.cu / sgmv.cu).
+int launch_plan_ids(lora_pool *pool, const int32_t *ids, int T, void *ws, cudaStream_t st);
+int launch_plan_segments(lora_pool *pool, const int32_t *off, const int32_t *slot, int S, int T,
+                         void *ws, cudaStream_t st);
+enum DecodeMode { kFused = 0, kShrinkOnly = 1, kExpandOnly = 2 };
+int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
+                  const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st);
+int decode_setup(lora_pool *pool);
+
+}  // namespace lora

@@ -1,0 +1,355 @@
+// pool.cu -- the paged adapter pool: slot layout, page free list, page table,
+// per-(slot, target) rank table, and the copy of adapter weights into pages.
+//
+// The pool follows the unified-paging idea of "Multi-LoRA Serving: Sharing One
+// GPU Across Adapters" (section "How S-LoRA Proved the Model"): adapter weights
+// live in fixed-size pages of one caller-provided buffer, located through a
+// page table, so adapters of any rank can come and go without fragmenting
+// device memory.  Every slot is padded to the pool's r_max (the static
+// max_lora_rank slot of "Multi-LoRA Serving: Why 100 Adapters Fit on One GPU",
+// section "Where does multi-LoRA serving actually break?", item 2).
+#include <algorithm>
+#include <cstring>
+#include <new>
+
+#include "internal.cuh"
+
+namespace lora {
+
+std::atomic<uint64_t> g_launches{0};
+
+static bool is_pow2(unsigned long long v) { return v && !(v & (v - 1)); }
+
+// Slot layout: per target an A block (r_max x d_in bf16) then a B^T block
+// (r_max x d_out bf16), each starting on a 256-byte boundary.
+static long long slot_layout(const lora_target *t, int n, int r_max, std::vector<long long> *a_off,
+                             std::vector<long long> *bt_off) {
+  long long off = 0;
+  for (int i = 0; i < n; ++i) {
+    if (a_off) a_off->push_back(off);
+    off += (long long)align256(size_t((long long)r_max * t[i].d_in * 2));
+    if (bt_off) bt_off->push_back(off);
+    off += (long long)align256(size_t((long long)r_max * t[i].d_out * 2));
+  }
+  return off;
+}
+
+static int check_shape(const lora_target *targets, int n_targets, int r_max, int n_slots, size_t page_bytes) {
+  if (!targets || n_targets < 1 || n_targets > kMaxTargets) return LORA_ERR_INVALID_ARG;
+  if (r_max < 1 || r_max > kRMax) return LORA_ERR_INVALID_ARG;
+  if (n_slots < 1 || n_slots > kMaxSlots) return LORA_ERR_INVALID_ARG;
+  if (page_bytes != 0 && (!is_pow2(page_bytes) || page_bytes < 4096)) return LORA_ERR_INVALID_ARG;
+  for (int i = 0; i < n_targets; ++i) {
+    if (targets[i].d_in < 8 || targets[i].d_out < 8) return LORA_ERR_INVALID_ARG;
+    if (targets[i].d_in > (1 << 20) || targets[i].d_out > (1 << 20)) return LORA_ERR_INVALID_ARG;
+    if ((targets[i].d_in % 8) || (targets[i].d_out % 8)) return LORA_ERR_ALIGNMENT;
+  }
+  return LORA_OK;
+}
+
+// splitmix64, used only to scatter the initial page order.
+static uint64_t splitmix64(uint64_t &s) {
+  uint64_t z = (s += 0x9E3779B97F4A7C15ull);
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Visit the physical pieces of a slot's logical byte range [off, off+bytes).
+template <class F>
+static void for_each_run(const lora_pool *p, int slot, long long off, long long bytes, F fn) {
+  long long done = 0;
+  while (done < bytes) {
+    long long page_idx = (p->pps == 1) ? 0 : (off + done) / p->page_bytes;
+    long long inside = (p->pps == 1) ? (off + done) : (off + done) % p->page_bytes;
+    long long n = std::min(bytes - done, p->page_bytes - inside);
+    int phys = p->pt[(size_t)slot * p->pps + page_idx];
+    fn(p->mem + (long long)phys * p->page_bytes + inside, done, n);
+    done += n;
+  }
+}
+
+// B (d_out x rank, row-major) -> rows j of B^T in the pool, through the page
+// table.  One thread per 8 consecutive output columns of one row j.
+__global__ void store_bt_kernel(PoolView pool, int slot, long long bt_off, int d_out, int rank,
+                                const uint16_t *B) {
+  long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  long long per_row = d_out / 8;
+  if (idx >= per_row * rank) return;
+  int j = (int)(idx / per_row);
+  int n0 = (int)(idx % per_row) * 8;
+  uint16_t v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = B[(long long)(n0 + e) * rank + j];
+  long long room;
+  const uint8_t *dst = pool_addr(pool, slot, bt_off + ((long long)j * d_out + n0) * 2, &room);
+  if (!dst) return;
+  uint4 packed;
+  packed.x = v[0] | (uint32_t(v[1]) << 16);
+  packed.y = v[2] | (uint32_t(v[3]) << 16);
+  packed.z = v[4] | (uint32_t(v[5]) << 16);
+  packed.w = v[6] | (uint32_t(v[7]) << 16);
+  *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(dst)) = packed;
+}
+
+}  // namespace lora
+
+using namespace lora;
+
+#define CUDA_TRY(expr)                            \
+  do {                                            \
+    if ((expr) != cudaSuccess) {                  \
+      (void)cudaGetLastError();                   \
+      return LORA_ERR_CUDA;                       \
+    }                                             \
+  } while (0)
+
+extern "C" {
+
+const char *lora_status_string(int s) {
+  switch (s) {
+    case LORA_OK: return "LORA_OK";
+    case LORA_ERR_INVALID_ARG: return "LORA_ERR_INVALID_ARG";
+    case LORA_ERR_ALIGNMENT: return "LORA_ERR_ALIGNMENT";
+    case LORA_ERR_NO_PAGES: return "LORA_ERR_NO_PAGES";
+    case LORA_ERR_SLOT: return "LORA_ERR_SLOT";
+    case LORA_ERR_NOT_LOADED: return "LORA_ERR_NOT_LOADED";
+    case LORA_ERR_CUDA: return "LORA_ERR_CUDA";
+    case LORA_ERR_BAD_ID: return "LORA_ERR_BAD_ID";
+    case LORA_ERR_TIMEOUT: return "LORA_ERR_TIMEOUT";
+    case LORA_ERR_WORKSPACE: return "LORA_ERR_WORKSPACE";
+    default: return "LORA_ERR_UNKNOWN";
+  }
+}
+
+size_t lora_pool_bytes_required(const lora_target *targets, int n_targets, int r_max, int n_slots,
+                                size_t page_bytes) {
+  if (check_shape(targets, n_targets, r_max, n_slots, page_bytes) != LORA_OK) return 0;
+  long long slot = slot_layout(targets, n_targets, r_max, nullptr, nullptr);
+  if (page_bytes == 0) return size_t(n_slots) * align256(size_t(slot));
+  long long pps = (slot + (long long)page_bytes - 1) / (long long)page_bytes;
+  return size_t(n_slots) * size_t(pps) * page_bytes;
+}
+
+int lora_pool_create(lora_pool **out, int device, const lora_target *targets, int n_targets, int r_max,
+                     int n_slots, size_t page_bytes, void *pool_mem, size_t pool_bytes,
+                     uint64_t scatter_seed) {
+  if (!out) return LORA_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = check_shape(targets, n_targets, r_max, n_slots, page_bytes);
+  if (rc != LORA_OK) return rc;
+  if (!pool_mem) return LORA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(pool_mem) & 255u) return LORA_ERR_ALIGNMENT;
+  int n_dev = 0;
+  CUDA_TRY(cudaGetDeviceCount(&n_dev));
+  if (device < 0 || device >= n_dev) return LORA_ERR_INVALID_ARG;
+
+  lora_pool *p = new (std::nothrow) lora_pool();
+  if (!p) return LORA_ERR_INVALID_ARG;
+  p->device = device;
+  p->n_targets = n_targets;
+  p->r_max = r_max;
+  p->n_slots = n_slots;
+  p->targets.assign(targets, targets + n_targets);
+  p->slot_bytes = slot_layout(targets, n_targets, r_max, &p->a_off, &p->bt_off);
+  if (page_bytes == 0) {
+    p->page_bytes = (long long)align256(size_t(p->slot_bytes));
+    p->pps = 1;
+    p->log2_page = -1;
+  } else {
+    p->page_bytes = (long long)page_bytes;
+    p->pps = (int)((p->slot_bytes + p->page_bytes - 1) / p->page_bytes);
+    int lg = 0;
+    while ((1ll << lg) < p->page_bytes) ++lg;
+    p->log2_page = (p->pps == 1) ? -1 : lg;
+  }
+  long long n_pages = (long long)(pool_bytes / (size_t)p->page_bytes);
+  if (n_pages < 1 || n_pages > (1ll << 31) - 1) {
+    delete p;
+    return LORA_ERR_INVALID_ARG;
+  }
+  p->n_pages = (int)n_pages;
+  p->mem = static_cast<uint8_t *>(pool_mem);
+  p->mem_bytes = pool_bytes;
+
+  // free list: ascending, or a seeded permutation; handed out from the front
+  std::vector<int32_t> order(p->n_pages);
+  for (int i = 0; i < p->n_pages; ++i) order[i] = i;
+  if (scatter_seed != 0) {
+    uint64_t s = scatter_seed;
+    for (int i = p->n_pages - 1; i > 0; --i) {
+      int j = (int)(splitmix64(s) % (uint64_t)(i + 1));
+      std::swap(order[i], order[j]);
+    }
+  }
+  p->free_pages.assign(order.rbegin(), order.rend());
+
+  p->pt.assign((size_t)n_slots * p->pps, -1);
+  p->rank.assign((size_t)n_slots * n_targets, 0);
+  p->loaded.assign((size_t)n_slots, 0);
+
+  DeviceGuard g(device);
+  size_t pt_b = align256(p->pt.size() * 4), rk_b = align256(p->rank.size() * 4),
+         ld_b = align256(p->loaded.size() * 4);
+  if (cudaMalloc(&p->dev_tables, pt_b + rk_b + ld_b + 256) != cudaSuccess) {
+    (void)cudaGetLastError();
+    delete p;
+    return LORA_ERR_CUDA;
+  }
+  uint8_t *b = static_cast<uint8_t *>(p->dev_tables);
+  p->d_pt = reinterpret_cast<int32_t *>(b);
+  p->d_rank = reinterpret_cast<int32_t *>(b + pt_b);
+  p->d_loaded = reinterpret_cast<int32_t *>(b + pt_b + rk_b);
+  p->d_status = reinterpret_cast<int *>(b + pt_b + rk_b + ld_b);
+  bool ok = cudaMemcpy(p->d_pt, p->pt.data(), p->pt.size() * 4, cudaMemcpyHostToDevice) == cudaSuccess &&
+            cudaMemset(p->d_rank, 0, p->rank.size() * 4) == cudaSuccess &&
+            cudaMemset(p->d_loaded, 0, p->loaded.size() * 4) == cudaSuccess &&
+            cudaMemset(p->d_status, 0, 4) == cudaSuccess && decode_setup(p) == LORA_OK;
+  if (!ok) {
+    (void)cudaGetLastError();
+    cudaFree(p->dev_tables);
+    delete p;
+    return LORA_ERR_CUDA;
+  }
+  *out = p;
+  return LORA_OK;
+}
+
+int lora_pool_load(lora_pool *p, int slot, int target, int rank, const void *A, const void *B,
+                   int src_is_device, void *stream) {
+  if (!p) return LORA_ERR_INVALID_ARG;
+  if (slot < 0 || slot >= p->n_slots) return LORA_ERR_SLOT;
+  if (target < 0 || target >= p->n_targets) return LORA_ERR_INVALID_ARG;
+  if (rank < 0 || rank > p->r_max) return LORA_ERR_INVALID_ARG;
+  if (rank > 0 && (!A || !B)) return LORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(p->mu);
+  DeviceGuard g(p->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int d_in = p->targets[target].d_in, d_out = p->targets[target].d_out;
+
+  if (!p->loaded[slot]) {
+    if ((int)p->free_pages.size() < p->pps) return LORA_ERR_NO_PAGES;
+    for (int i = 0; i < p->pps; ++i) {
+      p->pt[(size_t)slot * p->pps + i] = p->free_pages.back();
+      p->free_pages.pop_back();
+    }
+    p->loaded[slot] = 1;
+    CUDA_TRY(cudaMemcpyAsync(p->d_pt + (size_t)slot * p->pps, p->pt.data() + (size_t)slot * p->pps,
+                             (size_t)p->pps * 4, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(p->d_loaded + slot, p->loaded.data() + slot, 4, cudaMemcpyHostToDevice, st));
+  }
+
+  const long long a_off = p->a_off[target], bt_off = p->bt_off[target];
+  const long long a_used = (long long)rank * d_in * 2, a_all = (long long)p->r_max * d_in * 2;
+  const long long b_used = (long long)rank * d_out * 2, b_all = (long long)p->r_max * d_out * 2;
+  const cudaMemcpyKind kind = src_is_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  int rc = LORA_OK;
+  auto copy = [&](const uint8_t *src) {
+    return [&, src](uint8_t *dst, long long done, long long n) {
+      if (rc == LORA_OK && cudaMemcpyAsync(dst, src + done, (size_t)n, kind, st) != cudaSuccess) rc = LORA_ERR_CUDA;
+    };
+  };
+  auto zero = [&](uint8_t *dst, long long, long long n) {
+    if (rc == LORA_OK && cudaMemsetAsync(dst, 0, (size_t)n, st) != cudaSuccess) rc = LORA_ERR_CUDA;
+  };
+  if (rank > 0) {
+    for_each_run(p, slot, a_off, a_used, copy(static_cast<const uint8_t *>(A)));
+    if (src_is_device) {
+      long long n = (long long)rank * (d_out / 8);
+      int threads = 256;
+      g_launches.fetch_add(1);
+      store_bt_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
+          p->view(), slot, bt_off, d_out, rank, static_cast<const uint16_t *>(B));
+      if (cudaGetLastError() != cudaSuccess) rc = LORA_ERR_CUDA;
+    } else {
+      const uint16_t *Bh = static_cast<const uint16_t *>(B);
+      std::vector<uint16_t> bt((size_t)rank * d_out);
+      for (int n = 0; n < d_out; ++n)
+        for (int j = 0; j < rank; ++j) bt[(size_t)j * d_out + n] = Bh[(size_t)n * rank + j];
+      for_each_run(p, slot, bt_off, b_used, copy(reinterpret_cast<const uint8_t *>(bt.data())));
+    }
+  }
+  if (a_all > a_used) for_each_run(p, slot, a_off + a_used, a_all - a_used, zero);
+  if (b_all > b_used) for_each_run(p, slot, bt_off + b_used, b_all - b_used, zero);
+  if (rc != LORA_OK) {
+    (void)cudaGetLastError();
+    return rc;
+  }
+  p->rank[(size_t)slot * p->n_targets + target] = rank;
+  CUDA_TRY(cudaMemcpyAsync(p->d_rank + (size_t)slot * p->n_targets + target,
+                           p->rank.data() + (size_t)slot * p->n_targets + target, 4,
+                           cudaMemcpyHostToDevice, st));
+  if (!src_is_device) CUDA_TRY(cudaStreamSynchronize(st));  // host staging buffers go out of scope
+  return LORA_OK;
+}
+
+int lora_pool_unload(lora_pool *p, int slot) {
+  if (!p) return LORA_ERR_INVALID_ARG;
+  if (slot < 0 || slot >= p->n_slots) return LORA_ERR_SLOT;
+  std::lock_guard<std::mutex> lk(p->mu);
+  if (!p->loaded[slot]) return LORA_ERR_NOT_LOADED;
+  DeviceGuard g(p->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  for (int i = p->pps - 1; i >= 0; --i) {
+    p->free_pages.push_back(p->pt[(size_t)slot * p->pps + i]);
+    p->pt[(size_t)slot * p->pps + i] = -1;
+  }
+  for (int t = 0; t < p->n_targets; ++t) p->rank[(size_t)slot * p->n_targets + t] = 0;
+  p->loaded[slot] = 0;
+  CUDA_TRY(cudaMemcpy(p->d_pt + (size_t)slot * p->pps, p->pt.data() + (size_t)slot * p->pps,
+                      (size_t)p->pps * 4, cudaMemcpyHostToDevice));
+  CUDA_TRY(cudaMemcpy(p->d_rank + (size_t)slot * p->n_targets, p->rank.data() + (size_t)slot * p->n_targets,
+                      (size_t)p->n_targets * 4, cudaMemcpyHostToDevice));
+  CUDA_TRY(cudaMemcpy(p->d_loaded + slot, p->loaded.data() + slot, 4, cudaMemcpyHostToDevice));
+  return LORA_OK;
+}
+
+int lora_pool_destroy(lora_pool *p) {
+  if (!p) return LORA_ERR_INVALID_ARG;
+  int rc = LORA_OK;
+  {
+    DeviceGuard g(p->device);
+    if (cudaDeviceSynchronize() != cudaSuccess) rc = LORA_ERR_CUDA;
+    if (p->dev_tables && cudaFree(p->dev_tables) != cudaSuccess) rc = LORA_ERR_CUDA;
+    (void)cudaGetLastError();
+  }
+  delete p;
+  return rc;
+}
+
+const int32_t *lora_pool_page_table(const lora_pool *p) { return p ? p->d_pt : nullptr; }
+
+int lora_pool_get_info(const lora_pool *p, lora_pool_info *info) {
+  if (!p || !info) return LORA_ERR_INVALID_ARG;
+  info->slot_bytes = (size_t)p->slot_bytes;
+  info->page_bytes = (size_t)p->page_bytes;
+  info->pages_per_slot = p->pps;
+  info->n_pages = p->n_pages;
+  info->free_pages = (int)p->free_pages.size();
+  info->n_slots = p->n_slots;
+  info->n_targets = p->n_targets;
+  info->r_max = p->r_max;
+  return LORA_OK;
+}
+
+int lora_pool_target_offsets(const lora_pool *p, int target, size_t *a_off, size_t *bt_off) {
+  if (!p || target < 0 || target >= p->n_targets || !a_off || !bt_off) return LORA_ERR_INVALID_ARG;
+  *a_off = (size_t)p->a_off[target];
+  *bt_off = (size_t)p->bt_off[target];
+  return LORA_OK;
+}
+
+uint64_t lora_kernel_launches(void) { return g_launches.load(); }
+
+int lora_get_error(lora_pool *p, int *device_status, void *stream) {
+  if (!p || !device_status) return LORA_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  CUDA_TRY(cudaMemcpy(&v, p->d_status, 4, cudaMemcpyDeviceToHost));
+  CUDA_TRY(cudaMemset(p->d_status, 0, 4));
+  *device_status = v;
+  return LORA_OK;
+}
+
+}  // extern "C"

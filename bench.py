@@ -1,0 +1,476 @@
+"""Benchmark of the multi-LoRA delta path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload q_proj|tiny|prefill|mlp|paged]
+
+Default workload (the metric's configuration): Llama-2-7B q_proj-shaped decode,
+d_in = d_out = 4096, rank 16 for all, 32 resident adapters in a contiguous
+stacked pool, 64 tokens with ids uniform over the 32 adapters, bf16 inputs,
+fp32 accumulation.  A step is one lora_apply call (plan kernel + fused
+shrink/expand kernel) over one batch.  Steps rotate over 64 independent buffer
+sets (pool, x, y, ids, workspace), > 4x the 126 MB L2, so every step reads its
+adapters and activations from HBM.
+
+Printed: one JSON line (rank 0).  value = tokens/s over all ranks; roofline =
+algorithmic bytes of the dominant kernel / its mean launch time (CUDA events
+on the launching stream) against the measured HBM copy bandwidth;
+cpu_baseline = the fp64 oracle on the host cores on a bounded sample; e2e =
+the same metric through the C ABI with pinned host buffers copied in and the
+result copied out inside the timed region.
+
+With N > 1 (torchrun) every rank runs an independent replica on its own
+batches (tokens are independent; the path has no data exchange): weak scaling,
+timed per rank with CUDA events and reduced with a max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LoRA-delta tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
+WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5}
+L2_BYTES = 126 * 2 ** 20
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def algorithmic_bytes(w, target: int, ids) -> int:
+    """Bytes the delta must move for one call: each distinct adapter's A and B
+    at its own rank, x of every adapted row, and y of every adapted row read
+    and written."""
+    d_in, d_out = w.targets[target]
+    act = ids[ids >= 0]
+    act = act[w.rank[act] > 0]
+    distinct = np.unique(act)
+    adapters = int(sum(int(w.rank[a]) * (d_in + d_out) * 2 for a in distinct))
+    return adapters + act.size * d_in * 2 + act.size * d_out * 4
+
+
+def traffic_from_profile(kernel_file: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_%s.txt" % workload)
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    kv = {}
+    for ln in lines:
+        if ":" in ln:
+            k, v = ln.split(":", 1)
+            kv[k.strip()] = v.strip()
+    src = open(os.path.join(ROOT, "adapter_deltas_b200", "csrc", kernel_file), "rb").read()
+    if kv.get("source_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    try:
+        return int(kv["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        pass
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU arms
+
+
+def time_oracle(w, target: int, min_seconds: float, threads: int):
+    """Run the oracle on whole batches until min_seconds passed; tokens/s."""
+    import oracle
+    slots = [int(s) for s in np.unique(w.ids[w.ids >= 0])]
+    adapters = {s: w.adapter(s, target) for s in slots}
+    x, y = w.x(target), w.y_in(target)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.lora_apply(x, y, w.ids, w.n_slots, adapters, w.alpha, threads=threads)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return n * w.T / el, n, el
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank: int, world: int):
+    """The oracle, timed on the host cores, on the same workload and metric."""
+    if rank != 0:
+        return
+    import synth
+    w = synth.config(WORKLOADS[args.workload])
+    threads = min(cpu_threads(), w.T)
+    for _ in range(args.warmup):
+        time_oracle(w, 0, 0.0, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle(w, 0, 0.0, threads)
+    el = time.perf_counter() - t0
+    value = args.steps * w.T / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.T, "seq_len": 1, "parallelism": "oracle on host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": "%d whole batches of %d tokens" % (args.steps, w.T)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def run_b200(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import adapter_deltas_b200 as L
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.config(WORKLOADS[args.workload], seed=1000 + WORKLOADS[args.workload] + 1000 * rank)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    scales_np = np.zeros(w.n_slots, np.float32)
+    nz = w.rank > 0
+    scales_np[nz] = (w.alpha[nz] / w.rank[nz]).astype(np.float32)
+    scales = torch.from_numpy(scales_np).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    if args.workload == "paged":
+        return run_paged(args, rank, world, dev, w, scales, bf16)
+
+    # one buffer set: pool (all slots loaded), x, y, ids, workspace
+    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
+    act_bytes = w.T * sum(d_in + d_out for d_in, d_out in w.targets) * 2
+    set_bytes = pool_bytes + act_bytes
+    n_sets = max(2, min(64, -(-4 * L2_BYTES // set_bytes)))
+    target = 0
+    adapters = {}
+    for s in range(w.n_slots):
+        if w.rank[s] > 0:
+            A, B = w.adapter(s, target)
+            adapters[s] = (bf16(A), bf16(B))
+    x0, y0 = bf16(w.x(target)), bf16(w.y_in(target))
+    ids0 = torch.from_numpy(w.ids).to(dev)
+    sets = []
+    for k in range(n_sets):
+        mem = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
+        pool = L.lora_pool_create(local_rank, w.targets, w.r_max, w.n_slots, w.page_bytes, mem, w.scatter_seed)
+        for s, (A, B) in adapters.items():
+            L.lora_pool_load(pool, s, target, int(w.rank[s]), A, B)
+        ws = torch.zeros(L.lora_workspace_bytes(pool, target, w.T), dtype=torch.uint8, device=dev)
+        sets.append(dict(pool=pool, x=x0.clone(), y=y0.clone(), ids=ids0.clone(), ws=ws))
+    torch.cuda.synchronize()
+
+    def step(k):
+        s = sets[k % n_sets]
+        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"], stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- timed region: K whole steps
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = L.lora_kernel_launches()
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for k in range(args.steps):
+            step(args.warmup + k)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    launches = L.lora_kernel_launches() - launches0
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = reduce_max(ms, world, dev)
+
+    # ---- dominant kernel alone: the fused shrink/expand launch on prebuilt plans
+    for s in sets:
+        L.lora_plan_ids(s["pool"], s["ids"], s["ws"], stream)
+    reps = max(args.steps, 3 * n_sets)
+    for k in range(n_sets):
+        s = sets[k]
+        L.lora_apply_plan(s["pool"], target, s["x"], s["y"], scales, s["ws"], stream)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for k in range(reps):
+        s = sets[k % n_sets]
+        L.lora_apply_plan(s["pool"], target, s["x"], s["y"], scales, s["ws"], stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kernel_ms = ev0.elapsed_time(ev1) / reps
+
+    # ---- end to end through the C ABI with pinned host buffers
+    xh = x0.cpu().pin_memory()
+    yh = y0.cpu().pin_memory()
+    idh = ids0.cpu().pin_memory()
+    yout = torch.empty_like(yh).pin_memory()
+    h2d = xh.numel() * 2 + yh.numel() * 2 + idh.numel() * 4
+    d2h = yout.numel() * 2
+
+    def e2e_step(k):
+        s = sets[k % n_sets]
+        s["x"].copy_(xh, non_blocking=True)
+        s["y"].copy_(yh, non_blocking=True)
+        s["ids"].copy_(idh, non_blocking=True)
+        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"], stream)
+        yout.copy_(s["y"], non_blocking=True)
+
+    for k in range(args.warmup):
+        e2e_step(k)
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for k in range(args.steps):
+        e2e_step(k)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(ev0.elapsed_time(ev1) / args.steps, world, dev)
+
+    for s in sets:
+        L.lora_pool_destroy(s["pool"])
+    if rank != 0:
+        return
+
+    peak, peak_kind = load_peaks()
+    alg = algorithmic_bytes(w, target, w.ids)
+    achieved = alg / (kernel_ms * 1e-3) / 1e9
+    tokens = w.T * world
+    line = {
+        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": tokens, "seq_len": 1,
+                   "parallelism": "replicas%d" % world if world > 1 else "single",
+                   "adapters_in_batch": int(np.unique(w.ids[w.ids >= 0]).size),
+                   "l2": "%d rotating buffer sets, %.0f MB > 4x L2" % (n_sets, n_sets * set_bytes / 1e6)},
+        "hbm_gbs_step": alg * world / (ms * 1e-3) / 1e9 / world,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": traffic_from_profile("sgmv.cu", args.workload),
+                     "kernel": "decode_kernel<fused>", "kernel_us": kernel_ms * 1e3,
+                     "algorithmic_bytes_per_launch": alg, "frac_of_8TBps_datasheet": achieved / 8000.0},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "delta_vs_base_w_read": (kernel_ms * 1e-3) / (sum(a * b for a, b in w.targets[:1]) * 2 / (peak * 1e9)),
+    }
+    if world == 1:
+        threads = min(cpu_threads(), w.T)
+        v, n, el = time_oracle(w, target, args.cpu_seconds, threads)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": "%d whole batches of %d tokens (%.1f s)" % (n, w.T, el)}
+    print(json.dumps(line), flush=True)
+
+
+def run_paged(args, rank, world, dev, w, scales, bf16):
+    """All 128 layer x projection deltas of one decode step over the 31.25 GiB
+    paged pool: one plan, then one lora_apply_plan per matrix."""
+    import torch
+
+    import adapter_deltas_b200 as L
+    T, n_t = w.T, len(w.targets)
+    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
+    mem = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
+    pool = L.lora_pool_create(dev.index, w.targets, w.r_max, w.n_slots, w.page_bytes, mem, w.scatter_seed)
+    active = [int(s) for s in w.active_slots]
+    w.prefetch(active, range(n_t))
+    for s in active:
+        for t in range(n_t):
+            A, B = w.adapter(s, t)
+            L.lora_pool_load(pool, s, t, int(w.rank[s]), bf16(A), bf16(B))
+    g = torch.Generator(device=dev).manual_seed(7)
+    fa = (torch.randn(16, 4096, generator=g, device=dev) / 64).to(torch.bfloat16)
+    fb = (torch.randn(4096, 16, generator=g, device=dev) * 0.14).to(torch.bfloat16)
+    for s in range(w.n_slots):
+        if s not in set(active):
+            for t in range(n_t):
+                L.lora_pool_load(pool, s, t, 16, fa, fb)
+    xs = [bf16(w.x(t)) for t in range(n_t)]
+    ys = [bf16(w.y_in(t)) for t in range(n_t)]
+    w.drop()
+    ids = torch.from_numpy(w.ids).to(dev)
+    ws = torch.zeros(L.lora_workspace_bytes(pool, 0, T), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        L.lora_plan_ids(pool, ids, ws, stream)
+        for t in range(n_t):
+            L.lora_apply_plan(pool, t, xs[t], ys[t], scales, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = L.lora_kernel_launches()
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    launches = L.lora_kernel_launches() - l0
+    ms = reduce_max(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    # kernel alone: the 128 applies without the plan
+    ev0.record(stream)
+    for _ in range(args.steps):
+        for t in range(n_t):
+            L.lora_apply_plan(pool, t, xs[t], ys[t], scales, ws, stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kernel_ms = ev0.elapsed_time(ev1) / (args.steps * n_t)
+    L.lora_pool_destroy(pool)
+    if rank != 0:
+        return
+    peak, peak_kind = load_peaks()
+    alg = algorithmic_bytes(w, 0, w.ids)
+    achieved = alg / (kernel_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": T * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": T * world, "seq_len": 1, "parallelism": "single",
+                   "deltas_per_step": n_t, "l2": "pool 31.25 GiB and 1 GiB of activations per step > L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": traffic_from_profile("sgmv.cu", "paged"),
+                     "kernel": "decode_kernel<fused>", "kernel_us": kernel_ms * 1e3,
+                     "algorithmic_bytes_per_launch": alg},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def reduce_max(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default="q_proj", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        if args.impl == "reference":
+            if rank != 0:
+                return
+        else:
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local_rank))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_b200(args, rank, world, local_rank)
+    finally:
+        if world > 1 and args.impl != "reference":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,286 @@
+/*
+ * lora.h -- C ABI of the B200 multi-LoRA delta library (liblora_b200.so).
+ *
+ * What the library computes, for every row t of a mixed batch whose adapter
+ * id a = ids[t] is not -1:
+ *
+ *     y[t, :] += (alpha_a / r_a) * B_a (A_a x[t, :])
+ *
+ * with A_a of shape r_a x d_in and B_a of shape d_out x r_a.  This is the
+ * per-request adapter term of y = xW + (x A_i) B_i (alpha / r) from "Multi-LoRA
+ * Serving: Why 100 Adapters Fit on One GPU" (section "Why can't you just merge
+ * LoRA weights into the base model?"), with the adapter shapes of section "How
+ * much memory does one LoRA adapter actually cost?" of the same page, and the
+ * column form W.x + (B.A).x of "Serving Many LoRA Adapters From One Base
+ * Model" (section "How it works").  xW is produced by the caller; the library
+ * adds the delta in place.  All adapters of a batch are handled by one launch,
+ * driven by an index vector (segmented gather, first page, section "How does
+ * one batch run 30 different adapters at once?").  Adapters live in a paged
+ * pool with a page table ("Multi-LoRA Serving: Sharing One GPU Across
+ * Adapters", section "How S-LoRA Proved the Model").
+ *
+ * Conventions for every call:
+ *  - Return value: LORA_OK (0) or one of the LORA_ERR_* codes below.  No C++
+ *    exception crosses this boundary.
+ *  - Pointers named "device" are device pointers owned by the caller (for
+ *    example torch tensor storage); the library never frees them.
+ *  - stream is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  Compute calls are asynchronous on that stream and never
+ *    synchronise the host, never allocate, and may be captured in a CUDA graph.
+ *  - bf16 tensors are row-major with a leading dimension (ld*) counted in
+ *    elements.  x, y, weights and workspace must be 16-byte aligned, and
+ *    d_in, d_out, ldx and ldy must be multiples of 8, else LORA_ERR_ALIGNMENT.
+ *  - x and y must not overlap.
+ *  - Errors found on the device (bad adapter ids, timed-out waits) do not
+ *    fault: the affected rows are left untouched and a sticky per-pool status
+ *    word records the first error; read it with lora_get_error.
+ */
+#ifndef LORA_B200_H
+#define LORA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LORA_API __attribute__((visibility("default")))
+#else
+#define LORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+
+enum {
+    LORA_OK = 0,
+    LORA_ERR_INVALID_ARG = 1,  /* null pointer, size out of range, bad enum   */
+    LORA_ERR_ALIGNMENT = 2,    /* pointer / leading dimension alignment       */
+    LORA_ERR_NO_PAGES = 3,     /* the page pool has too few free pages        */
+    LORA_ERR_SLOT = 4,         /* slot index out of range                     */
+    LORA_ERR_NOT_LOADED = 5,   /* slot holds no adapter (host check, or sticky
+                                  device status when a batch names it)        */
+    LORA_ERR_CUDA = 6,         /* a CUDA runtime call failed                  */
+    LORA_ERR_BAD_ID = 7,       /* sticky device status: an id outside
+                                  [-1, n_slots) or a malformed segment        */
+    LORA_ERR_TIMEOUT = 8,      /* sticky device status: a bounded wait inside
+                                  a kernel gave up                            */
+    LORA_ERR_WORKSPACE = 9     /* workspace smaller than lora_workspace_bytes */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+LORA_API const char *lora_status_string(int status);
+
+/* ------------------------------------------------------------- the pool */
+
+/* Opaque pool handle; allocated by lora_pool_create, freed by
+ * lora_pool_destroy.  It owns small device tables (page table, ranks, status
+ * word) but not the page memory, which the caller provides. */
+typedef struct lora_pool lora_pool;
+
+/* One adapted weight matrix (a layer's projection): W is d_out x d_in. */
+typedef struct {
+    int d_in;
+    int d_out;
+} lora_target;
+
+/*
+ * Slot layout (the logical bytes of one adapter slot).  Targets follow one
+ * another in order.  Target t holds A (r_max rows of d_in bf16; row j is
+ * adapter row j) and then B transposed (r_max rows of d_out bf16; row j is
+ * column j of B).  Each of these two blocks starts on a 256-byte boundary.
+ * Rows rank..r_max-1 of both blocks are zero (rank padding, the static
+ * max_lora_rank slot of "Multi-LoRA Serving: Why 100 Adapters Fit on One GPU",
+ * section "Where does multi-LoRA serving actually break?", item 2); kernels
+ * read only the adapter's own rank.
+ *
+ * Paging.  A slot's logical bytes are cut into pages of page_bytes; page p of
+ * slot s lives at physical page page_table[s * pages_per_slot + p], i.e. at
+ * byte pool_mem + page * page_bytes.  page_bytes == 0 means one page per slot
+ * (a contiguous stacked pool [n_slots][slot_bytes rounded up to 256]).
+ */
+
+/* Bytes of page memory needed to hold every slot at once (0 on bad args).
+ * page_bytes: 0, or a power of two >= 4096. */
+LORA_API size_t lora_pool_bytes_required(const lora_target *targets, int n_targets,
+                                int r_max, int n_slots, size_t page_bytes);
+
+/*
+ * Create a pool over caller-owned device memory.
+ *   device        CUDA device ordinal the pool and all its calls use.
+ *   targets       n_targets (1..4096) matrix shapes, copied.
+ *   r_max         rank of a slot (1..64).
+ *   n_slots       number of adapter slots (1..16384).
+ *   page_bytes    0 (one page per slot) or a power of two >= 4096.
+ *   pool_mem      device buffer of pool_bytes bytes, 256-byte aligned; it may
+ *                 hold fewer pages than n_slots need (pages are taken from a
+ *                 free list when a slot is first loaded: LORA_ERR_NO_PAGES when
+ *                 it runs out).
+ *   scatter_seed  0: free pages in ascending order; otherwise a seeded
+ *                 permutation, so a slot's pages are scattered over the pool.
+ * Returns LORA_OK and *out, or an error (nothing allocated).
+ */
+LORA_API int lora_pool_create(lora_pool **out, int device, const lora_target *targets,
+                     int n_targets, int r_max, int n_slots, size_t page_bytes,
+                     void *pool_mem, size_t pool_bytes, uint64_t scatter_seed);
+
+/*
+ * Copy one adapter matrix pair into a slot.
+ *   rank   the adapter's rank on this target, 0..r_max (0 marks the target as
+ *          not adapted: rows of this slot are then left untouched on it).
+ *   A      bf16 [rank, d_in], row-major, dense.
+ *   B      bf16 [d_out, rank], row-major, dense; stored transposed.
+ *   src_is_device  1: A and B are device pointers (copies are asynchronous on
+ *          stream); 0: host pointers (the call returns once the host data has
+ *          been staged; the device copies complete in stream order).
+ * The first load into an empty slot takes its pages from the free list.
+ * Loading must not race with compute calls that read the same slot.
+ */
+LORA_API int lora_pool_load(lora_pool *pool, int slot, int target, int rank,
+                   const void *A, const void *B, int src_is_device,
+                   void *stream);
+
+/* Release a slot's pages to the free list and mark it empty (its rows then
+ * raise LORA_ERR_NOT_LOADED).  Synchronous with respect to the device. */
+LORA_API int lora_pool_unload(lora_pool *pool, int slot);
+
+/* Free the pool's own device tables and the handle (not pool_mem).  Waits for
+ * the device. */
+LORA_API int lora_pool_destroy(lora_pool *pool);
+
+/* Device pointer to the page table, int32 [n_slots][pages_per_slot]; -1 marks
+ * a page that is not allocated.  Read-only; valid until destroy. */
+LORA_API const int32_t *lora_pool_page_table(const lora_pool *pool);
+
+/* Geometry of a pool, for callers that walk its memory (tests, tools). */
+typedef struct {
+    size_t slot_bytes;      /* logical bytes of one slot                     */
+    size_t page_bytes;      /* physical page size (one slot when 0 was given) */
+    int pages_per_slot;
+    int n_pages;            /* physical pages in pool_mem                    */
+    int free_pages;
+    int n_slots, n_targets, r_max;
+} lora_pool_info;
+
+LORA_API int lora_pool_get_info(const lora_pool *pool, lora_pool_info *info);
+
+/* Byte offsets inside a slot of target t's A block and B-transposed block. */
+LORA_API int lora_pool_target_offsets(const lora_pool *pool, int target,
+                             size_t *a_off, size_t *bt_off);
+
+/* ---------------------------------------------------------- the workspace */
+
+/*
+ * Device workspace for batches of up to max_tokens rows (the call's T): holds
+ * the plan (rows grouped by adapter, work items).  The target argument is
+ * accepted for future per-target needs; the size does not depend on it today.
+ */
+LORA_API size_t lora_workspace_bytes(const lora_pool *pool, int target, int max_tokens);
+
+/* Where each plan array lives inside a workspace sized for T rows (byte
+ * offsets from the workspace base). */
+typedef struct {
+    size_t header;      /* int32[64]: [0] segments, [1] rows grouped,
+                           [2] decode work items, [3] tensor-core tiles,
+                           [4] T                                          */
+    size_t perm;        /* int32[T]: row indices grouped by segment        */
+    size_t seg_start;   /* int32[S_max+1]: segment s = perm[seg_start[s] ..
+                           seg_start[s+1])                                 */
+    size_t seg_slot;    /* int32[S_max]: slot of segment s                 */
+    size_t items;       /* int32[I_max][4]: decode items {slot, first perm
+                           index, rows, segment}                            */
+    size_t tiles;       /* int32[J_max][4]: tensor-core tiles {slot, first
+                           row of x/y, rows, segment}                       */
+    size_t total;
+    int s_max, i_max, j_max;
+} lora_plan_layout;
+
+LORA_API int lora_plan_layout_get(const lora_pool *pool, int T, lora_plan_layout *out);
+
+/* ---------------------------------------------------------------- plans */
+
+/*
+ * Build the plan of a batch from its index vector: rows grouped by adapter
+ * (segments in ascending slot order, rows in ascending order inside a
+ * segment), split into work items.  ids: device int32 [T], -1 = no adapter.
+ * Rows with an invalid id (outside [-1, n_slots): LORA_ERR_BAD_ID; an empty
+ * slot: LORA_ERR_NOT_LOADED) join no segment and set the sticky status.
+ * A plan depends only on the batch, so one plan serves every target of a
+ * forward step (lora_apply_plan).
+ */
+LORA_API int lora_plan_ids(lora_pool *pool, const int32_t *ids, int T, void *ws,
+                  size_t ws_bytes, void *stream);
+
+/*
+ * Build the plan of a batch given as contiguous segments: rows
+ * seg_offsets[s] .. seg_offsets[s+1]-1 use slot seg_slot[s].
+ *   seg_offsets  device int32 [S+1], non-decreasing, within [0, T];
+ *   seg_slot     device int32 [S]; -1 = the segment has no adapter.
+ * Segments at least lora_mma_min_rows() long take the tensor-core path; the
+ * others the decode path.  Malformed segments are skipped (LORA_ERR_BAD_ID).
+ */
+LORA_API int lora_plan_segments(lora_pool *pool, const int32_t *seg_offsets,
+                       const int32_t *seg_slot, int S, int T, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/* Segment length from which the tensor-core path is used. */
+LORA_API int lora_mma_min_rows(void);
+
+/*
+ * Apply a built plan to one target:  y[t] += scales[a] * B_a (A_a x[t]).
+ *   x       device bf16 [T, ldx] (ldx >= d_in)
+ *   y       device bf16 [T, ldy] (ldy >= d_out), updated in place: each
+ *           adapted element becomes bf16_rn(y + scale * delta) computed in
+ *           fp32; other rows are not touched.
+ *   scales  device fp32 [n_slots]: alpha / r of each slot's adapter.
+ *   T, ws, ws_bytes  as passed to the plan call.
+ */
+LORA_API int lora_apply_plan(lora_pool *pool, int target, const void *x, int ldx,
+                    void *y, int ldy, const float *scales, int T,
+                    const void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------- one-call entry */
+
+/* lora_plan_ids followed by lora_apply_plan. */
+LORA_API int lora_apply(lora_pool *pool, int target, const void *x, int ldx, void *y,
+               int ldy, const int32_t *ids, const float *scales, int T,
+               void *ws, size_t ws_bytes, void *stream);
+
+/* lora_plan_segments followed by lora_apply_plan. */
+LORA_API int lora_apply_segments(lora_pool *pool, int target, const void *x, int ldx,
+                        void *y, int ldy, const int32_t *seg_offsets,
+                        const int32_t *seg_slot, int S, const float *scales,
+                        int T, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The two halves of the delta, for callers that keep v = A_a x[t]:
+ *   lora_shrink writes v[t, 0:r_max] (fp32, device [T, ldv], ldv >= r_max;
+ *   entries r_a..r_max-1 are written as 0) for every row with an adapter,
+ *   and leaves other rows of v untouched.
+ *   lora_expand adds scales[a] * B_a v[t, 0:r_a] to y[t] in place.
+ * lora_shrink followed by lora_expand gives bit-identical y to lora_apply:
+ * both use the same reduction order.
+ */
+LORA_API int lora_shrink(lora_pool *pool, int target, const void *x, int ldx,
+                const int32_t *ids, int T, float *v, int ldv, void *ws,
+                size_t ws_bytes, void *stream);
+
+LORA_API int lora_expand(lora_pool *pool, int target, const float *v, int ldv, void *y,
+                int ldy, const int32_t *ids, const float *scales, int T,
+                void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------ diagnostics */
+
+/* Synchronise stream, then read and clear the pool's sticky device status
+ * (LORA_OK when no device-side error happened since the last read). */
+LORA_API int lora_get_error(lora_pool *pool, int *device_status, void *stream);
+
+/* Number of kernels this library has launched in this process. */
+LORA_API uint64_t lora_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_B200_H */
