@@ -49,7 +49,8 @@ class lora_target(ctypes.Structure):
 
 class lora_pool_info(ctypes.Structure):
     _fields_ = [("slot_bytes", _Z), ("page_bytes", _Z), ("pages_per_slot", _I), ("n_pages", _I),
-                ("free_pages", _I), ("n_slots", _I), ("n_targets", _I), ("r_max", _I)]
+                ("free_pages", _I), ("n_slots", _I), ("n_targets", _I), ("r_max", _I),
+                ("decode_clusters", _I)]
 
 
 class lora_plan_layout(ctypes.Structure):

@@ -329,6 +329,7 @@ int lora_pool_get_info(const lora_pool *p, lora_pool_info *info) {
   info->n_slots = p->n_slots;
   info->n_targets = p->n_targets;
   info->r_max = p->r_max;
+  info->decode_clusters = p->decode_max_clusters;
   return LORA_OK;
 }
 

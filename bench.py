@@ -209,8 +209,6 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     nz = w.rank > 0
     scales_np[nz] = (w.alpha[nz] / w.rank[nz]).astype(np.float32)
     scales = torch.from_numpy(scales_np).to(dev)
-    stream = torch.cuda.current_stream(dev)
-
     if args.workload == "paged":
         return run_paged(args, rank, world, dev, w, scales, bf16)
 
@@ -239,46 +237,47 @@ def run_b200(args, rank: int, world: int, local_rank: int):
 
     def step(k):
         s = sets[k % n_sets]
-        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"], stream)
+        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"])
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    # ---- timed region: K whole steps
-    for k in range(args.warmup):
-        step(k)
+    # ---- timed region: a CUDA graph of exactly K whole steps
+    g_warm, _ = capture_graph(dev, step, range(args.warmup))
+    g_main, launches = capture_graph(dev, step, range(args.warmup, args.warmup + args.steps))
+    g_warm.replay()
     torch.cuda.synchronize()
     barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = L.lora_kernel_launches()
     sampler = ClockSampler(local_rank)
     with sampler:
         torch.cuda.synchronize()
-        ev0.record(stream)
-        for k in range(args.steps):
-            step(args.warmup + k)
-        ev1.record(stream)
+        ev0.record()
+        g_main.replay()
+        ev1.record()
         torch.cuda.synchronize()
     clocks = sampler.stop()
-    launches = L.lora_kernel_launches() - launches0
     barrier()
     ms = ev0.elapsed_time(ev1) / args.steps
     ms = reduce_max(ms, world, dev)
 
     # ---- dominant kernel alone: the fused shrink/expand launch on prebuilt plans
     for s in sets:
-        L.lora_plan_ids(s["pool"], s["ids"], s["ws"], stream)
+        L.lora_plan_ids(s["pool"], s["ids"], s["ws"])
     reps = max(args.steps, 3 * n_sets)
-    for k in range(n_sets):
-        s = sets[k]
-        L.lora_apply_plan(s["pool"], target, s["x"], s["y"], scales, s["ws"], stream)
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    for k in range(reps):
+
+    def apply_only(k):
         s = sets[k % n_sets]
-        L.lora_apply_plan(s["pool"], target, s["x"], s["y"], scales, s["ws"], stream)
-    ev1.record(stream)
+        L.lora_apply_plan(s["pool"], target, s["x"], s["y"], scales, s["ws"])
+
+    g_kw, _ = capture_graph(dev, apply_only, range(n_sets))
+    g_k, _ = capture_graph(dev, apply_only, range(reps))
+    g_kw.replay()
+    torch.cuda.synchronize()
+    ev0.record()
+    g_k.replay()
+    ev1.record()
     torch.cuda.synchronize()
     kernel_ms = ev0.elapsed_time(ev1) / reps
 
@@ -295,19 +294,20 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         s["x"].copy_(xh, non_blocking=True)
         s["y"].copy_(yh, non_blocking=True)
         s["ids"].copy_(idh, non_blocking=True)
-        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"], stream)
+        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"])
         yout.copy_(s["y"], non_blocking=True)
 
-    for k in range(args.warmup):
-        e2e_step(k)
+    g_ew, _ = capture_graph(dev, e2e_step, range(args.warmup))
+    g_e, _ = capture_graph(dev, e2e_step, range(args.steps))
+    g_ew.replay()
     torch.cuda.synchronize()
     barrier()
-    ev0.record(stream)
-    for k in range(args.steps):
-        e2e_step(k)
-    ev1.record(stream)
+    ev0.record()
+    g_e.replay()
+    ev1.record()
     torch.cuda.synchronize()
     e2e_ms = reduce_max(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    del g_warm, g_main, g_kw, g_k, g_ew, g_e
 
     for s in sets:
         L.lora_pool_destroy(s["pool"])
@@ -325,7 +325,8 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         "config": {"workload": w.name, "global_batch": tokens, "seq_len": 1,
                    "parallelism": "replicas%d" % world if world > 1 else "single",
                    "adapters_in_batch": int(np.unique(w.ids[w.ids >= 0]).size),
-                   "l2": "%d rotating buffer sets, %.0f MB > 4x L2" % (n_sets, n_sets * set_bytes / 1e6)},
+                   "l2": "%d rotating buffer sets, %.0f MB > 4x L2" % (n_sets, n_sets * set_bytes / 1e6),
+                   "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "hbm_gbs_step": alg * world / (ms * 1e-3) / 1e9 / world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
@@ -374,36 +375,38 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
     w.drop()
     ids = torch.from_numpy(w.ids).to(dev)
     ws = torch.zeros(L.lora_workspace_bytes(pool, 0, T), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
-    def step():
-        L.lora_plan_ids(pool, ids, ws, stream)
+    def step(_k):
+        L.lora_plan_ids(pool, ids, ws)
         for t in range(n_t):
-            L.lora_apply_plan(pool, t, xs[t], ys[t], scales, ws, stream)
+            L.lora_apply_plan(pool, t, xs[t], ys[t], scales, ws)
 
-    for _ in range(args.warmup):
-        step()
+    g_warm, _ = capture_graph(dev, step, range(args.warmup))
+    g_main, launches = capture_graph(dev, step, range(args.steps))
+    g_warm.replay()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    l0 = L.lora_kernel_launches()
     sampler = ClockSampler(dev.index)
     with sampler:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
+        ev0.record()
+        g_main.replay()
+        ev1.record()
         torch.cuda.synchronize()
     clocks = sampler.stop()
-    launches = L.lora_kernel_launches() - l0
     ms = reduce_max(ev0.elapsed_time(ev1) / args.steps, world, dev)
+
     # kernel alone: the 128 applies without the plan
-    ev0.record(stream)
-    for _ in range(args.steps):
+    def applies(_k):
         for t in range(n_t):
-            L.lora_apply_plan(pool, t, xs[t], ys[t], scales, ws, stream)
-    ev1.record(stream)
+            L.lora_apply_plan(pool, t, xs[t], ys[t], scales, ws)
+
+    g_k, _ = capture_graph(dev, applies, range(args.steps))
+    ev0.record()
+    g_k.replay()
+    ev1.record()
     torch.cuda.synchronize()
     kernel_ms = ev0.elapsed_time(ev1) / (args.steps * n_t)
+    del g_warm, g_main, g_k
     L.lora_pool_destroy(pool)
     if rank != 0:
         return
@@ -415,7 +418,8 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": T * world, "seq_len": 1, "parallelism": "single",
-                   "deltas_per_step": n_t, "l2": "pool 31.25 GiB and 1 GiB of activations per step > L2"},
+                   "deltas_per_step": n_t, "l2": "pool 31.25 GiB and 1 GiB of activations per step > L2",
+                   "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind, "traffic": traffic_from_profile("sgmv.cu", "paged"),
                      "kernel": "decode_kernel<fused>", "kernel_us": kernel_ms * 1e3,
@@ -423,6 +427,25 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
         "gpu_launches": launches, "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def capture_graph(dev, fn, ks):
+    """Capture fn(k) for k in ks into one CUDA graph; also return how many of
+    the library's kernels the captured calls launch."""
+    import torch
+
+    import adapter_deltas_b200 as L
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    n0 = L.lora_kernel_launches()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for k in ks:
+                fn(k)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    return g, L.lora_kernel_launches() - n0
 
 
 def reduce_max(x: float, world: int, dev) -> float:

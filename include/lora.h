@@ -161,6 +161,8 @@ typedef struct {
     int n_pages;            /* physical pages in pool_mem                    */
     int free_pages;
     int n_slots, n_targets, r_max;
+    int decode_clusters;    /* thread-block clusters of the decode kernel
+                               that can be resident at once on this device */
 } lora_pool_info;
 
 LORA_API int lora_pool_get_info(const lora_pool *pool, lora_pool_info *info);
