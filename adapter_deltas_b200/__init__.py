@@ -84,6 +84,7 @@ _sig("lora_apply", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_segments", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_shrink", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
+_sig("lora_apply_noalloc", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
 _sig("lora_get_error", _I, [_P, ctypes.POINTER(_I), _P])
 _sig("lora_kernel_launches", ctypes.c_uint64, [])
 
@@ -258,6 +259,17 @@ def lora_shrink(pool: PoolHandle, target: int, x, ids, v, ws, stream=None) -> No
 def lora_expand(pool: PoolHandle, target: int, v, y, ids, scales, ws, stream=None) -> None:
     _check(_lib.lora_expand(pool, target, _ptr(v), _ld(v), _ptr(y), _ld(y), _ptr(ids), _ptr(scales),
                             ids.shape[0], _ptr(ws), ws.numel(), _stream(stream)), "lora_expand")
+
+
+LORA_NOALLOC_MAX_TOKENS = 4096
+
+
+def lora_apply_noalloc(pool: PoolHandle, target: int, x, y, ids, scales, stream=None) -> None:
+    """lora_apply without a workspace argument: the plan lives in a fixed
+    device array inside the library (for callers that cannot allocate).
+    Calls that overlap on the GPU share that array and must be serialised."""
+    _check(_lib.lora_apply_noalloc(pool, target, _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(ids), _ptr(scales),
+                                   y.shape[0], _stream(stream)), "lora_apply_noalloc")
 
 
 def lora_get_error(pool: PoolHandle, stream=None) -> int:

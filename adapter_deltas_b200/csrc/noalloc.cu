@@ -1,0 +1,75 @@
+// noalloc.cu -- lora_apply for callers that cannot allocate device memory.
+//
+// lora_apply needs a workspace for the batch plan.  Some callers cannot hand
+// one over: their device memory belongs to an allocator they must not bypass
+// (a framework's caching allocator, a serving runtime that pre-sizes every
+// buffer), or they run in a loop that may not take the implicit device
+// synchronisation cudaMalloc and cudaFree can cause.  lora_apply_noalloc keeps
+// the plan in a fixed array compiled into this library instead.  Every GPU
+// that loads the library holds that array until the process exits.
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace lora {
+namespace {
+
+// Plan bytes for LORA_NOALLOC_MAX_TOKENS rows (an upper bound of
+// plan_layout(LORA_NOALLOC_MAX_TOKENS).total; each call checks the exact size).
+constexpr size_t kNoAllocT = LORA_NOALLOC_MAX_TOKENS;
+constexpr size_t kNoAllocBytes = 8 * 256 + 4 * kNoAllocT * 4 + 4 * 4 +
+                                 (kNoAllocT + kNoAllocT / kItemRows + 1) * 16 +
+                                 ((3 * kNoAllocT + kMmaRows - 1) / kMmaRows + 1) * 16;
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on `device` (which must be current).
+// The first call on a device looks it up; later calls reuse it.
+int scratch_address(int device, void **out) {
+  if (device < 0 || device >= kMaxDevices) return LORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_scratch_addr[device]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      (void)cudaGetLastError();
+      return LORA_ERR_CUDA;
+    }
+    g_scratch_addr[device] = ptr;
+  }
+  *out = g_scratch_addr[device];
+  return LORA_OK;
+}
+
+}  // namespace
+}  // namespace lora
+
+using namespace lora;
+
+extern "C" int lora_apply_noalloc(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
+                                  const int32_t *ids, const float *scales, int T, void *stream) {
+  if (!p || target < 0 || target >= p->n_targets || T < 0) return LORA_ERR_INVALID_ARG;
+  if (T == 0) return LORA_OK;
+  const size_t need = plan_layout(T).total;
+  if (T > LORA_NOALLOC_MAX_TOKENS || need > kNoAllocBytes) return LORA_ERR_WORKSPACE;
+  if (!x || !y || !ids || !scales) return LORA_ERR_INVALID_ARG;
+  const int d_in = p->targets[target].d_in, d_out = p->targets[target].d_out;
+  if (ldx < d_in || ldy < d_out) return LORA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || (ldx % 8) || (ldy % 8)) return LORA_ERR_ALIGNMENT;
+  const char *xa = static_cast<const char *>(x), *ya = static_cast<const char *>(y);
+  if (xa < ya + size_t(T) * ldy * 2 && ya < xa + size_t(T) * ldx * 2) return LORA_ERR_INVALID_ARG;
+
+  DeviceGuard g(p->device);
+  void *ws = nullptr;
+  int rc = scratch_address(p->device, &ws);
+  if (rc != LORA_OK) return rc;
+  // Nothing in the scratch needs clearing: the plan kernel rewrites every word
+  // the delta kernel then reads (header counts, segments, items, rows).
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = launch_plan_ids(p, ids, T, ws, st);
+  if (rc != LORA_OK) return rc;
+  return launch_decode(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st);
+}

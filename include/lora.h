@@ -272,6 +272,39 @@ LORA_API int lora_expand(lora_pool *pool, int target, const float *v, int ldv, v
                 int ldy, const int32_t *ids, const float *scales, int T,
                 void *ws, size_t ws_bytes, void *stream);
 
+/* ------------------------------------------------- no-allocation variant */
+
+/* Largest batch (T) that lora_apply_noalloc accepts. */
+#define LORA_NOALLOC_MAX_TOKENS 4096
+
+/*
+ * lora_apply for callers that cannot allocate device memory.  The web pages
+ * this library follows have no counterpart of this call; it exists because
+ * some callers cannot provide the plan workspace that lora_apply takes: their
+ * device memory is owned by an allocator they must not go around (a
+ * framework's caching allocator, a serving runtime that sizes every buffer up
+ * front), or they run in a loop that cannot afford the device-wide
+ * synchronisation that cudaMalloc / cudaFree may cause.
+ *
+ * The call computes exactly what lora_apply computes, with the same
+ * arguments minus ws / ws_bytes.  The plan lives in one fixed array of device
+ * memory compiled into the library (138,800 bytes, enough for
+ * LORA_NOALLOC_MAX_TOKENS rows); every GPU that loads the library holds that
+ * array until the process exits.  The call itself allocates nothing.
+ *   - T > LORA_NOALLOC_MAX_TOKENS returns LORA_ERR_WORKSPACE (nothing runs).
+ *   - The first call on a device looks up the array's device address (a
+ *     runtime query, done once per device with that device current); make
+ *     that first call before capturing a stream into a CUDA graph.
+ *   - All calls share the one array, which keeps the last call's plan.  No
+ *     part of it needs clearing (each call rewrites everything it reads), but
+ *     calls that overlap on the GPU -- on different streams, or on different
+ *     pools of the same device -- race on it and must be serialised by the
+ *     caller.
+ */
+LORA_API int lora_apply_noalloc(lora_pool *pool, int target, const void *x, int ldx, void *y,
+                                int ldy, const int32_t *ids, const float *scales, int T,
+                                void *stream);
+
 /* ------------------------------------------------------------ diagnostics */
 
 /* Synchronise stream, then read and clear the pool's sticky device status
