@@ -34,6 +34,19 @@ bool overlap(const void *x, int ldx, const void *y, int ldy, int T) {
   return xa < yb && ya < xb;
 }
 
+enum { kPlanUnknown = 0, kPlanIds = 1, kPlanSegments = 2 };
+
+void set_plan_kind(lora_pool *p, const void *ws, int kind) {
+  std::lock_guard<std::mutex> lk(p->mu);
+  p->plan_kind[ws] = kind;
+}
+
+int plan_kind(lora_pool *p, const void *ws) {
+  std::lock_guard<std::mutex> lk(p->mu);
+  auto it = p->plan_kind.find(ws);
+  return it == p->plan_kind.end() ? kPlanUnknown : it->second;
+}
+
 }  // namespace
 
 extern "C" {
@@ -66,7 +79,9 @@ int lora_plan_ids(lora_pool *p, const int32_t *ids, int T, void *ws, size_t ws_b
   if (rc != LORA_OK || T == 0) return rc;
   if (!ids) return LORA_ERR_INVALID_ARG;
   DeviceGuard g(p->device);
-  return launch_plan_ids(p, ids, T, ws, static_cast<cudaStream_t>(stream));
+  rc = launch_plan_ids(p, ids, T, ws, static_cast<cudaStream_t>(stream));
+  if (rc == LORA_OK) set_plan_kind(p, ws, kPlanIds);
+  return rc;
 }
 
 int lora_plan_segments(lora_pool *p, const int32_t *seg_offsets, const int32_t *seg_slot, int S, int T, void *ws,
@@ -77,7 +92,9 @@ int lora_plan_segments(lora_pool *p, const int32_t *seg_offsets, const int32_t *
   if (T == 0) return LORA_OK;
   if (S > 0 && (!seg_offsets || !seg_slot)) return LORA_ERR_INVALID_ARG;
   DeviceGuard g(p->device);
-  return launch_plan_segments(p, seg_offsets, seg_slot, S, T, ws, static_cast<cudaStream_t>(stream));
+  rc = launch_plan_segments(p, seg_offsets, seg_slot, S, T, ws, static_cast<cudaStream_t>(stream));
+  if (rc == LORA_OK) set_plan_kind(p, ws, kPlanSegments);
+  return rc;
 }
 
 int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const float *scales, int T,
@@ -89,8 +106,19 @@ int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, i
   if (!scales) return LORA_ERR_INVALID_ARG;
   if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
   DeviceGuard g(p->device);
-  return launch_decode(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws,
-                       static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int kind = plan_kind(p, ws);
+  if (kind == kPlanIds)  // index-vector plans hold decode items only
+    return launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItems);
+  PrefillGeometry geo;
+  if (kind == kPlanSegments && prefill_geometry(p, target, &geo)) {
+    // short segments on the decode kernel, long ones on the tensor cores
+    rc = launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItems);
+    if (rc != LORA_OK) return rc;
+    return launch_prefill(p, target, x, ldx, y, ldy, scales, T, ws, st);
+  }
+  // every segment on the decode kernel
+  return launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItemsAll);
 }
 
 int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const int32_t *ids,

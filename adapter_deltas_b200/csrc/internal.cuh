@@ -11,6 +11,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "lora.h"
@@ -26,7 +27,7 @@ constexpr int kItemRows = 16;        // rows per decode work item
 constexpr int kTileVecs = 32;        // 16-byte vectors per pipeline tile row (512 B)
 constexpr int kTileRowBytes = kTileVecs * 16;
 constexpr int kMmaRows = 128;        // rows per tensor-core tile
-constexpr int kMmaMinRows = 1 << 30; // segment length that selects the tensor-core path
+constexpr int kMmaMinRows = 64;     // segment length that selects the tensor-core path
 constexpr int kPlanThreads = 1024;
 constexpr int kDecodeThreads = 256;
 constexpr int kClusterCtas = 8;      // CTAs that split one work item (portable cluster)
@@ -93,7 +94,10 @@ inline PlanLayout plan_layout(int T) {
 }
 
 // Header words of a plan.
-enum { kHdrSegs = 0, kHdrActive = 1, kHdrItems = 2, kHdrTiles = 3, kHdrT = 4 };
+// kHdrItemsAll counts the decode items of every segment, long ones included
+// (they follow the short segments' items), for targets the tensor-core path
+// cannot serve.
+enum { kHdrSegs = 0, kHdrActive = 1, kHdrItems = 2, kHdrTiles = 3, kHdrT = 4, kHdrItemsAll = 5 };
 
 struct PlanView {
   int32_t *hdr;
@@ -226,6 +230,10 @@ struct lora_pool {
   int *d_status = nullptr;
   int decode_smem = 0;
   int decode_max_clusters = 0;
+  // Kind of the plan last built into each workspace (1 = index vector,
+  // 2 = segments, which may hold tensor-core tiles); kept on the host so that
+  // an apply call can pick its kernels without reading the device.
+  std::unordered_map<const void *, int> plan_kind;
   std::mutex mu;
 
   lora::PoolView view() const {
@@ -266,6 +274,15 @@ int launch_plan_segments(lora_pool *pool, const int32_t *off, const int32_t *slo
 enum DecodeMode { kFused = 0, kShrinkOnly = 1, kExpandOnly = 2 };
 int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
                   const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st);
+int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
+                        const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
+                        int items_hdr);
+struct PrefillGeometry {
+  int C, nsx, nsy, r_cap, ks_cols, ns_cols, smem;
+};
+bool prefill_geometry(const lora_pool *pool, int target, PrefillGeometry *g);
+int launch_prefill(lora_pool *pool, int target, const void *x, int ldx, void *y, int ldy, const float *scales,
+                   int T, const void *ws, cudaStream_t st);
 int decode_setup(lora_pool *pool);
 
 }  // namespace lora

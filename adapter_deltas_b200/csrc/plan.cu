@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_ids_kernel(const int32_t *_
     plan.hdr[kHdrItems] = carry.c;
     plan.hdr[kHdrTiles] = 0;
     plan.hdr[kHdrT] = T;
+    plan.hdr[kHdrItemsAll] = carry.c;
   }
   __syncthreads();
 
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
       plan.hdr[kHdrItems] = 0;
       plan.hdr[kHdrTiles] = 0;
       plan.hdr[kHdrT] = T;
+      plan.hdr[kHdrItemsAll] = 0;
       set_status(status, LORA_ERR_BAD_ID);
     }
     return;
@@ -191,6 +193,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
       }
     }
     const bool mma = len >= mma_min;
+    // c: decode items of short segments; d: tiles of long segments
     Quad v = {len, len > 0 ? 1 : 0, (len > 0 && !mma) ? (len + kItemRows - 1) / kItemRows : 0,
               mma ? (len + kMmaRows - 1) / kMmaRows : 0};
     Quad tot;
@@ -212,6 +215,18 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
     }
     carry = quad_add(carry, tot);
   }
+  __syncthreads();
+  // Decode items for the long segments too (after the short ones): targets
+  // the tensor-core path cannot serve take every segment on the decode path.
+  // Each tile of kMmaRows rows becomes kMmaRows / kItemRows items.
+  const int n_tiles = carry.d, n_short = carry.c;
+  for (int idx = tid; idx < n_tiles * (kMmaRows / kItemRows); idx += kPlanThreads) {
+    const int j = idx / (kMmaRows / kItemRows), q = idx - j * (kMmaRows / kItemRows);
+    const int4 t = plan.tiles[j];
+    const int first = t.y - plan.seg_row[t.w] + plan.seg_start[t.w] + q * kItemRows;  // perm index
+    const int m = min(kItemRows, t.z - q * kItemRows);
+    plan.items[n_short + idx] = m > 0 ? make_int4(t.x, first, m, t.w) : make_int4(t.x, first, 0, t.w);
+  }
   if (tid == 0) {
     plan.seg_start[carry.b] = carry.a;
     plan.hdr[kHdrSegs] = carry.b;
@@ -219,6 +234,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
     plan.hdr[kHdrItems] = carry.c;
     plan.hdr[kHdrTiles] = carry.d;
     plan.hdr[kHdrT] = T;
+    plan.hdr[kHdrItemsAll] = n_short + n_tiles * (kMmaRows / kItemRows);
   }
   __syncthreads();
   // perm: the rows of segment g are seg_row[g] .. seg_row[g] + length - 1

@@ -50,6 +50,7 @@ struct DecodeArgs {
   long long ldv;
   int *status;
   int stage_bytes;
+  int items_hdr;  // header word holding the item count to process
 };
 
 // Copy `bytes` of slot's logical range starting at `off` into dst, cut at
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
   __syncthreads();
   griddep_wait();
 
-  const int n_items = a.hdr[kHdrItems];
+  const int n_items = a.hdr[a.items_hdr];
   const int nvi = a.d_in / 8, nvo = a.d_out / 8;
   const int per_i = (nvi + C - 1) / C, per_o = (nvo + C - 1) / C;
   const int kv0 = min(crank * per_i, nvi), kv1 = min(kv0 + per_i, nvi);
@@ -232,7 +233,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
     const int t_idx = shrink ? tt : tt - nk;
     const int v_lo = (shrink ? kv0 : nv0) + t_idx * kTileVecs;
     const int wv = max(0, min(v_lo + kTileVecs, shrink ? kv1 : nv1) - v_lo);
-    const int rows = (wv > 0 && r > 0) ? r + m : 0;
+    const int rows = (wv > 0 && r > 0 && m > 0) ? r + m : 0;
     const uint32_t row_bytes = (uint32_t)wv * 16u;
     if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)rows * row_bytes);
     __syncwarp();
@@ -285,11 +286,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
     __syncthreads();
     const int jb = r <= 8 ? 1 : r <= 16 ? 2 : r <= 32 ? 4 : 8;
     for (int tt = 0; tt < tpi; ++tt, ++g) {
-      if (MODE == kFused && tt == nk && r > 0) exchange(m, r);
+      if (MODE == kFused && tt == nk && r > 0 && m > 0) exchange(m, r);
       const int stage = (int)(g % kStages);
       const uint32_t parity = (uint32_t)((g / kStages) & 1);
       const bool ok = mbar_wait_bounded(&full[stage], parity, a.status);
-      if (ok && r > 0) {
+      if (ok && r > 0 && m > 0) {
         const uint8_t *buf = ring + stage * a.stage_bytes;
         const bool shrink = tt < nk;
         const int t_idx = shrink ? tt : tt - nk;
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
       __syncthreads();  // stage consumed by every thread
       if (warp == 0 && g + kStages < total_tiles) issue(g + kStages);
     }
-    if (MODE == kShrinkOnly && r > 0) {
+    if (MODE == kShrinkOnly && r > 0 && m > 0) {
       exchange(m, r);
       if (crank == 0) {
         for (int idx = tid; idx < m * a.r_max; idx += kDecodeThreads) {
@@ -379,6 +380,12 @@ int decode_setup(lora_pool *pool) {
 
 int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
                   const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st) {
+  return launch_decode_items(pool, mode, target, x, ldx, y, ldy, scales, v, ldv, T, ws, st, kHdrItems);
+}
+
+int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
+                        const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
+                        int items_hdr) {
   PlanLayout L = plan_layout(T);
   PlanView pv = plan_view(const_cast<void *>(ws), L);
   DecodeArgs a;
@@ -400,6 +407,7 @@ int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx,
   a.v = v;
   a.ldv = ldv;
   a.status = pool->d_status;
+  a.items_hdr = items_hdr;
   int stage;
   const int smem = decode_smem_bytes(pool->r_max, &stage);
   a.stage_bytes = stage;

@@ -184,8 +184,10 @@ LORA_API size_t lora_workspace_bytes(const lora_pool *pool, int target, int max_
  * offsets from the workspace base). */
 typedef struct {
     size_t header;      /* int32[64]: [0] segments, [1] rows grouped,
-                           [2] decode work items, [3] tensor-core tiles,
-                           [4] T                                          */
+                           [2] decode work items of the segments on the
+                           decode path, [3] tensor-core tiles, [4] T,
+                           [5] decode items when every segment takes the
+                           decode path (long segments' items follow)     */
     size_t perm;        /* int32[T]: row indices grouped by segment        */
     size_t seg_start;   /* int32[S_max+1]: segment s = perm[seg_start[s] ..
                            seg_start[s+1])                                 */
@@ -219,8 +221,11 @@ LORA_API int lora_plan_ids(lora_pool *pool, const int32_t *ids, int T, void *ws,
  * seg_offsets[s] .. seg_offsets[s+1]-1 use slot seg_slot[s].
  *   seg_offsets  device int32 [S+1], non-decreasing, within [0, T];
  *   seg_slot     device int32 [S]; -1 = the segment has no adapter.
- * Segments at least lora_mma_min_rows() long take the tensor-core path; the
- * others the decode path.  Malformed segments are skipped (LORA_ERR_BAD_ID).
+ * Segments at least lora_mma_min_rows() long take the tensor-core path (in
+ * 128-row tiles) when the target allows it (r_max <= 32 and the slices fit in
+ * shared memory), the others the decode path.  Offsets that decrease or leave
+ * [0, T] make the whole plan empty (LORA_ERR_BAD_ID); segments naming an
+ * invalid slot are skipped (LORA_ERR_BAD_ID / LORA_ERR_NOT_LOADED).
  */
 LORA_API int lora_plan_segments(lora_pool *pool, const int32_t *seg_offsets,
                        const int32_t *seg_slot, int S, int T, void *ws,

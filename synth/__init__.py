@@ -10,6 +10,7 @@ from .workloads import (  # noqa: F401
     Workload,
     bf16_bits_to_f32,
     config,
+    custom,
     f32_to_bf16_bits,
     integer_case,
     normal_bf16,

@@ -283,3 +283,16 @@ def integer_case(seed: int, T: int, d_in: int, d_out: int, ranks: Sequence[int],
         ids = _rng(seed, _T_IDS).integers(-1, n, size=T)
     return Workload("integer case", seed, [(d_in, d_out)], r_max, n, page_bytes, scatter_seed,
                     T, np.asarray(ids, dtype=np.int32), rank, alpha, value_mode="integer")
+
+
+def custom(seed: int, T: int, targets: Sequence[Tuple[int, int]], ranks: Sequence[int], r_max: int,
+           alpha: Optional[Sequence[float]] = None, ids: Optional[Sequence[int]] = None,
+           y_mode: str = "normal", page_bytes: int = 0, scatter_seed: int = 0) -> Workload:
+    """A workload with the standard value recipe and caller-chosen geometry
+    (alpha defaults to 2 r, ids to uniform over the slots)."""
+    rank = np.array(ranks, dtype=np.int32)
+    a = 2.0 * rank.astype(np.float64) if alpha is None else np.asarray(alpha, dtype=np.float64)
+    if ids is None:
+        ids = _rng(seed, _T_IDS).integers(0, len(ranks), size=T)
+    return Workload("custom", seed, list(targets), r_max, len(ranks), page_bytes, scatter_seed, T,
+                    np.asarray(ids, dtype=np.int32), rank, a, y_mode=y_mode)
