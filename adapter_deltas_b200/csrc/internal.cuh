@@ -24,14 +24,16 @@ constexpr int kMaxSlots = 16384;     // plan kernel keeps one counter per slot i
 constexpr int kMaxTargets = 4096;
 constexpr int kMaxTokens = 1 << 20;
 constexpr int kItemRows = 16;        // rows per decode work item
-constexpr int kTileVecs = 32;        // 16-byte vectors per pipeline tile row (512 B)
-constexpr int kTileRowBytes = kTileVecs * 16;
+
 constexpr int kMmaRows = 128;        // rows per tensor-core tile
 constexpr int kMmaMinRows = 64;     // segment length that selects the tensor-core path
 constexpr int kPlanThreads = 1024;
-constexpr int kDecodeThreads = 256;
+constexpr int kConsumerWarps = 8;    // decode kernel: 8 warps, each copies and computes
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kDecodeThreads = kConsumerThreads;
 constexpr int kClusterCtas = 8;      // CTAs that split one work item (portable cluster)
-constexpr int kStages = 4;           // pipeline depth of the decode kernel
+constexpr int kMaxStages = 4;        // pipeline depth of the decode kernel
+constexpr int kItemSlots = 8;        // items a warp's copies may run ahead of its compute
 
 extern std::atomic<uint64_t> g_launches;
 

@@ -24,13 +24,10 @@
 // fixed CTA order, so every CTA ends with the same fp32 v (deterministic, and
 // independent of the other rows of the batch).  The expand then adds
 // scale * (B v) to its y slice in fp32 and stores bf16 (round to nearest even).
-#include <cooperative_groups.h>
-
 #include <algorithm>
 
 #include "internal.cuh"
 
-namespace cg = cooperative_groups;
 
 namespace lora {
 
@@ -50,6 +47,9 @@ struct DecodeArgs {
   long long ldv;
   int *status;
   int stage_bytes;
+  int n_stages;
+  int tile_vecs;  // 16-byte vectors per staged row (64 or 32)
+  int row_pitch;  // bytes between staged rows (tile_vecs * 16 + 16)
   int items_hdr;  // header word holding the item count to process
 };
 
@@ -73,265 +73,546 @@ __device__ __forceinline__ void copy_pool_row(const PoolView &pool, int slot, lo
   }
 }
 
-// Reduce JB per-lane values over the 32 lanes of a warp.  After the call
-// acc[0] of lane l holds the full sum of value index (l >> (5 - log2 JB)).
+// Shrink, output-stationary.  Lane l owns rank j = l % RW of the adapter
+// (and j + 32 when the slot rank exceeds 32) and the rows i = l / RW (mod NH)
+// of the item, RW = min(8 JB, 32) lanes per row phase, NH = 32 / RW phases.
+// Warp w takes the 16-byte column vectors w, w + 8, ... of every tile, so the
+// K dimension is split over the warps (and over the cluster's CTAs), and each
+// lane accumulates complete dot products of its outputs in registers for the
+// whole item: no cross-lane reduction.  The warps' partial sums are added in
+// shared memory once per item.
 template <int JB>
-__device__ __forceinline__ void warp_reduce_multi(float (&acc)[JB], int lane) {
-  int off = 16;
-#pragma unroll
-  for (int n = JB; n > 1; n >>= 1, off >>= 1) {
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int q = 0; q < n / 2; ++q) {
-      const float send = upper ? acc[q] : acc[q + n / 2];
-      const float keep = upper ? acc[q + n / 2] : acc[q];
-      acc[q] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-#pragma unroll
-  for (; off >= 1; off >>= 1) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
-}
-
-template <int JB>
-struct Log2 {
-  static constexpr int v = JB == 1 ? 0 : JB == 2 ? 1 : JB == 4 ? 2 : 3;
+struct ShrinkShape {
+  static constexpr int RW = JB * 8 < 32 ? JB * 8 : 32;  // lanes sharing one row phase
+  static constexpr int NH = 32 / RW;                     // row phases
+  static constexpr int NJ = JB * 8 > 32 ? 2 : 1;         // ranks per lane
+  static constexpr int NU = kItemRows / NH;              // rows per lane
+  static constexpr int NACC = NU * NJ;
 };
 
-// One shrink tile: columns [v_lo*8, v_lo*8 + wv*8) of the item's rows.  Warp w
-// owns adapter rows j = w + 8q (q < JB); lane l owns the l-th 16-byte column
-// vector.  Partial dot products accumulate into s_part[i][j] (this CTA's
-// share of v), each (i, j) written by exactly one lane.
 template <int JB>
-__device__ __forceinline__ void shrink_tile(const uint8_t *buf, int act_base, int wv, int r, int m,
-                                            float *s_part, int lane, int warp) {
-  if (warp >= r) return;
-  float a[JB][8];
+__device__ __forceinline__ void shrink_accumulate(const uint8_t *buf, int act_base, int pitch, int wv, int r, int m,
+                                                  float (&acc)[ShrinkShape<JB>::NACC], int lane, int warp) {
+  using SS = ShrinkShape<JB>;
+  const int jl = lane % SS::RW, ih = lane / SS::RW;
+  for (int kv = warp; kv < wv; kv += kConsumerWarps) {
+    float av[SS::NJ][8];
 #pragma unroll
-  for (int q = 0; q < JB; ++q) {
-    const int j = warp + 8 * q;
-    if (j < r && lane < wv) {
-      unpack8(*reinterpret_cast<const uint4 *>(buf + j * kTileRowBytes + lane * 16), a[q]);
-    } else {
+    for (int h = 0; h < SS::NJ; ++h) {
+      const int j = jl + 32 * h;
+      if (j < r) {
+        unpack8(*reinterpret_cast<const uint4 *>(buf + j * pitch + kv * 16), av[h]);
+      } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a[q][e] = 0.f;
+        for (int e = 0; e < 8; ++e) av[h][e] = 0.f;
+      }
     }
-  }
-  const uint8_t *xb = buf + act_base;
-  const int own_q = lane >> (5 - Log2<JB>::v);
-  const bool writer = (lane & ((32 / JB) - 1)) == 0;
-  for (int i = 0; i < m; ++i) {
-    float xv[8];
-    if (lane < wv) {
-      unpack8(*reinterpret_cast<const uint4 *>(xb + i * kTileRowBytes + lane * 16), xv);
-    } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xv[e] = 0.f;
+    for (int u = 0; u < SS::NU; ++u) {
+      const int i = ih + SS::NH * u;
+      if (i < m) {
+        float xv[8];
+        unpack8(*reinterpret_cast<const uint4 *>(buf + act_base + i * pitch + kv * 16), xv);
+#pragma unroll
+        for (int h = 0; h < SS::NJ; ++h) {
+          float s0 = acc[u * SS::NJ + h], s1 = av[h][1] * xv[1];
+          s0 = fmaf(av[h][0], xv[0], s0);
+          s1 = fmaf(av[h][3], xv[3], s1);
+          s0 = fmaf(av[h][2], xv[2], s0);
+          s1 = fmaf(av[h][5], xv[5], s1);
+          s0 = fmaf(av[h][4], xv[4], s0);
+          s1 = fmaf(av[h][7], xv[7], s1);
+          s0 = fmaf(av[h][6], xv[6], s0);
+          acc[u * SS::NJ + h] = s0 + s1;
+        }
+      }
     }
-    float acc[JB];
-#pragma unroll
-    for (int q = 0; q < JB; ++q) {
-      float s = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s = fmaf(a[q][e], xv[e], s);
-      acc[q] = s;
-    }
-    warp_reduce_multi<JB>(acc, lane);
-    const int j = warp + 8 * own_q;
-    if (writer && j < r) s_part[i * kRMax + j] += acc[0];
   }
 }
 
-// One expand tile: columns [v_lo*8, v_lo*8 + wv*8) of d_out.  Warp w owns rows
-// w and w + 8 of the item; lane l owns the l-th 16-byte column vector.
-__device__ __forceinline__ void expand_tile(const uint8_t *buf, int act_base, int wv, int v_lo, int r, int m,
-                                            const float *s_v, float scale, const int *s_rows,
-                                            const DecodeArgs &a, int lane, int warp) {
-  if (warp >= m || lane >= wv) return;
-  const bool two = warp + 8 < m;
-  float acc0[8], acc1[8];
+// This warp's partial sums of the item -> red[warp][i * r + j].
+template <int JB>
+__device__ __forceinline__ void shrink_spill(const float (&acc)[ShrinkShape<JB>::NACC], int r, int m, float *red,
+                                             int lane) {
+  using SS = ShrinkShape<JB>;
+  const int jl = lane % SS::RW, ih = lane / SS::RW;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    acc0[e] = 0.f;
-    acc1[e] = 0.f;
-  }
-  const float *v0 = s_v + warp * kRMax;
-  const float *v1 = s_v + (warp + 8) * kRMax;
-  for (int j = 0; j < r; ++j) {
-    float b[8];
-    unpack8(*reinterpret_cast<const uint4 *>(buf + j * kTileRowBytes + lane * 16), b);
-    const float c0 = v0[j];
+  for (int u = 0; u < SS::NU; ++u) {
+    const int i = ih + SS::NH * u;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc0[e] = fmaf(c0, b[e], acc0[e]);
-    if (two) {
-      const float c1 = v1[j];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc1[e] = fmaf(c1, b[e], acc1[e]);
+    for (int h = 0; h < SS::NJ; ++h) {
+      const int j = jl + 32 * h;
+      if (i < m && j < r) red[i * r + j] = acc[u * SS::NJ + h];
     }
-  }
-  const uint8_t *yb = buf + act_base;
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    if (rr == 1 && !two) break;
-    const int i = warp + 8 * rr;
-    float yv[8];
-    unpack8(*reinterpret_cast<const uint4 *>(yb + i * kTileRowBytes + lane * 16), yv);
-    const float *acc = rr ? acc1 : acc0;
-    uint4 o;
-    o.x = pack_bf16x2(fmaf(scale, acc[0], yv[0]), fmaf(scale, acc[1], yv[1]));
-    o.y = pack_bf16x2(fmaf(scale, acc[2], yv[2]), fmaf(scale, acc[3], yv[3]));
-    o.z = pack_bf16x2(fmaf(scale, acc[4], yv[4]), fmaf(scale, acc[5], yv[5]));
-    o.w = pack_bf16x2(fmaf(scale, acc[6], yv[6]), fmaf(scale, acc[7], yv[7]));
-    const long long row = s_rows[i];
-    *reinterpret_cast<uint4 *>(a.y + row * a.ldy + (long long)(v_lo + lane) * 8) = o;
   }
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs a) {
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = (int)cluster.num_blocks();
-  const int crank = (int)cluster.block_rank();
-  const int cid = blockIdx.x / C;
-  const int ncl = gridDim.x / C;
+// One expand tile: columns [v_lo*8, v_lo*8 + wv*8) of d_out.  Work units are
+// (group of RT rows, 4 consecutive columns), spread over all threads of the
+// CTA; a unit walks the ranks 4 at a time (loads first, then FMAs), so every
+// B vector it loads serves its RT rows.  RT = 4 for items of more than four
+// rows, else 1.
+template <int RT>
+__device__ __forceinline__ void expand_units(const uint8_t *buf, int act_base, int pitch, int wv, int v_lo, int r, int m,
+                                             const float *s_v, float scale, const int *s_rows, const DecodeArgs &a,
+                                             int tid) {
+  const int n4 = 2 * wv;                 // 4-column units per row
+  const int groups = (m + RT - 1) / RT;
+  for (int idx = tid; idx < groups * n4; idx += kConsumerThreads) {
+    const int gi = idx / n4, c4 = idx - gi * n4;
+    float acc[RT][4];
+#pragma unroll
+    for (int k = 0; k < RT; ++k)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
+    const uint8_t *bcol = buf + c4 * 8;
+    for (int j0 = 0; j0 < r; j0 += 4) {
+      float b[4][4], c[RT][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u;
+        if (j < r) {
+          const uint2 q = *reinterpret_cast<const uint2 *>(bcol + j * pitch);
+          b[u][0] = bf16_lo(q.x);
+          b[u][1] = bf16_hi(q.x);
+          b[u][2] = bf16_lo(q.y);
+          b[u][3] = bf16_hi(q.y);
+#pragma unroll
+          for (int k = 0; k < RT; ++k) c[k][u] = s_v[(gi * RT + k) * kRMax + j];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) b[u][e] = 0.f;
+#pragma unroll
+          for (int k = 0; k < RT; ++k) c[k][u] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int k = 0; k < RT; ++k)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[k][e] = fmaf(c[k][u], b[u][e], acc[k][e]);
+    }
+#pragma unroll
+    for (int k = 0; k < RT; ++k) {
+      const int i = gi * RT + k;
+      if (i < m) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(buf + act_base + i * pitch + c4 * 8);
+        uint2 o;
+        o.x = pack_bf16x2(fmaf(scale, acc[k][0], bf16_lo(u.x)), fmaf(scale, acc[k][1], bf16_hi(u.x)));
+        o.y = pack_bf16x2(fmaf(scale, acc[k][2], bf16_lo(u.y)), fmaf(scale, acc[k][3], bf16_hi(u.y)));
+        *reinterpret_cast<uint2 *>(a.y + (long long)s_rows[i] * a.ldy + (long long)v_lo * 8 + c4 * 4) = o;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void expand_tile(const uint8_t *buf, int act_base, int pitch, int wv, int v_lo, int r,
+                                            int m, const float *s_v, float scale, const int *s_rows,
+                                            const DecodeArgs &a, int tid) {
+  if (m <= 4)
+    expand_units<1>(buf, act_base, pitch, wv, v_lo, r, m, s_v, scale, s_rows, a, tid);
+  else
+    expand_units<4>(buf, act_base, pitch, wv, v_lo, r, m, s_v, scale, s_rows, a, tid);
+}
+
+// ------------------------------------------------------------ cluster helpers
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t addr, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(cta));
+  return r;
+}
+// Asynchronous 4-byte store into a peer CTA's shared memory that signals the
+// peer's mbarrier with its byte count on arrival.
+__device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (data written by peer CTAs).
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity, int *status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 255u) == 255u && global_timer_ns() - t0 > kSpinNs) break;
+  }
+  atomicCAS(status, 0, LORA_ERR_TIMEOUT);
+  return false;
+}
+// Per-lane 16-byte asynchronous copy global -> shared (L2 only), and an
+// arrive on an mbarrier once all of this thread's prior copies have landed.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src));
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier of the consumer warps only (named barrier 1).
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
+
+// Per-item facts a warp needs while it consumes an item.  Every warp keeps
+// its own copy (it resolved the item itself when it began copying it), so no
+// warp waits on another to learn what it is computing.
+struct ItemInfo {
+  int m, r;
+  float scale;
+  int pad;
+  int rows[kItemRows];
+};
+
+struct DecodeSmem {
+  uint8_t *ring;
+  uint64_t *full, *empty, *recv_full;
+  ItemInfo *info;  // [kConsumerWarps][kItemSlots]
+  float *red;      // [kConsumerWarps][kItemRows * r_max]: the warps' shrink partials
+  float *v, *recv;
+};
+
+__device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeArgs &a) {
+  DecodeSmem S;
+  uint8_t *p = smem;
+  S.ring = p; p += a.n_stages * a.stage_bytes;
+  S.full = reinterpret_cast<uint64_t *>(p); p += kMaxStages * 8;
+  S.empty = reinterpret_cast<uint64_t *>(p); p += kMaxStages * 8;
+  S.recv_full = reinterpret_cast<uint64_t *>(p); p += 2 * 8;
+  S.info = reinterpret_cast<ItemInfo *>(p); p += kConsumerWarps * kItemSlots * sizeof(ItemInfo);
+  S.red = reinterpret_cast<float *>(p); p += kConsumerWarps * kItemRows * a.r_max * 4;
+  S.v = reinterpret_cast<float *>(p); p += kItemRows * kRMax * 4;
+  S.recv = reinterpret_cast<float *>(p);  // [2][C][kItemRows * r_max]
+  return S;
+}
+
+// Where a warp's next copies come from: the item it is copying, with the
+// addresses of its rows held by the lanes (lane L: weight rows L and L + 32,
+// activation row L).
+struct IssueState {
+  int li, tt;
+  int slot, m, r;
+  bool split_a, split_b;
+  unsigned long long wa0, wa1, wb0, wb1, xrow, yrow;
+  int4 d_next;
+};
+
+template <int MODE, int JB>
+__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeArgs a) {
+  const int C = (int)cluster_nctarank();
+  const int crank = (int)cluster_ctarank();
+  const int cid = blockIdx.x / C, ncl = gridDim.x / C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int NS = a.n_stages;
 
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t *ring = smem;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * a.stage_bytes);
-  float *s_part = reinterpret_cast<float *>(full + kStages);
-  float *s_v = s_part + kItemRows * kRMax;
-  int *s_rows = reinterpret_cast<int *>(s_v + kItemRows * kRMax);
-  const int act_base = a.r_max * kTileRowBytes;  // activation rows follow r_max weight rows
+  const DecodeSmem S = decode_carve(smem, a);
+  ItemInfo *my_info = S.info + warp * kItemSlots;
+  const int TV = a.tile_vecs, pitch = a.row_pitch;
+  const int act_base = a.r_max * pitch;  // activation rows follow r_max weight rows
+  const int recv_slice = kItemRows * a.r_max;    // floats one source CTA may send per item
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&S.full[s], kConsumerThreads);  // every lane arrives once its copies of the tile landed
+      mbar_init(&S.empty[s], kConsumerWarps);   // every warp arrives once it is done with the tile
+    }
+    mbar_init(&S.recv_full[0], 1);
+    mbar_init(&S.recv_full[1], 1);
     fence_mbar_init();
   }
   __syncthreads();
+  // Peers may push into this CTA's shared memory only after its barriers are
+  // initialised: arrive now, wait before the first push.
+  cluster_arrive_relaxed();
   griddep_wait();
 
+  // the header and this cluster's first item are read together (the items
+  // array always has room for cid, whatever the count)
   const int n_items = a.hdr[a.items_hdr];
+  const int4 d0 = a.items[cid];
   const int nvi = a.d_in / 8, nvo = a.d_out / 8;
   const int per_i = (nvi + C - 1) / C, per_o = (nvo + C - 1) / C;
   const int kv0 = min(crank * per_i, nvi), kv1 = min(kv0 + per_i, nvi);
   const int nv0 = min(crank * per_o, nvo), nv1 = min(nv0 + per_o, nvo);
-  const int nk = (MODE == kExpandOnly) ? 0 : (per_i + kTileVecs - 1) / kTileVecs;
-  const int nn = (MODE == kShrinkOnly) ? 0 : (per_o + kTileVecs - 1) / kTileVecs;
+  const int nk = (MODE == kExpandOnly) ? 0 : (per_i + TV - 1) / TV;
+  const int nn = (MODE == kShrinkOnly) ? 0 : (per_o + TV - 1) / TV;
   const int tpi = nk + nn;
   const int my_items = cid < n_items ? (n_items - cid + ncl - 1) / ncl : 0;
-  const long long total_tiles = (long long)my_items * tpi;
+  const int total = my_items * tpi;
+  const int wlen_a = (kv1 - kv0) * 16, wlen_b = (nv1 - nv0) * 16;
 
-  // Producer: warp 0 fills ring stage g % kStages with tile g.
-  auto issue = [&](long long g) {
-    const int li = (int)(g / tpi), tt = (int)(g % tpi);
-    const int4 d = a.items[cid + li * ncl];
-    const int slot = d.x, pbeg = d.y, m = d.z;
-    const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
-    const int stage = (int)(g % kStages);
-    uint8_t *buf = ring + stage * a.stage_bytes;
-    const bool shrink = tt < nk;
-    const int t_idx = shrink ? tt : tt - nk;
-    const int v_lo = (shrink ? kv0 : nv0) + t_idx * kTileVecs;
-    const int wv = max(0, min(v_lo + kTileVecs, shrink ? kv1 : nv1) - v_lo);
-    const int rows = (wv > 0 && r > 0 && m > 0) ? r + m : 0;
-    const uint32_t row_bytes = (uint32_t)wv * 16u;
-    if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)rows * row_bytes);
+  // ---- resolve an item: one level of loads after the item record, all
+  // issued together; lane L keeps the addresses of rows L / L + 32 of this
+  // CTA's weight slices and of activation row L.
+  IssueState is;
+  is.li = 0;
+  is.tt = 0;
+  is.d_next = d0;
+  auto resolve = [&](int li) {
+    const int4 d = is.d_next;
+    if (li + 1 < my_items) is.d_next = a.items[cid + (li + 1) * ncl];  // lands while this item streams
+    is.slot = d.x;
+    is.m = d.z;
+    is.r = a.pool.rank[is.slot * a.pool.n_targets + a.target];
+    const float scale = a.scales ? a.scales[is.slot] : 0.f;
+    const int my_row = lane < is.m ? a.perm[d.y + lane] : 0;
+    const uint8_t *wa[2] = {nullptr, nullptr}, *wb[2] = {nullptr, nullptr};
+    bool sa = false, sb = false;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = lane + 32 * h;
+      if (j < a.r_max) {
+        long long room;
+        if (MODE != kExpandOnly && wlen_a > 0) {
+          wa[h] = pool_addr(a.pool, is.slot, a.a_off + ((long long)j * a.d_in + (long long)kv0 * 8) * 2, &room);
+          sa |= (j < is.r) && (wa[h] == nullptr || room < wlen_a);
+        }
+        if (MODE != kShrinkOnly && wlen_b > 0) {
+          wb[h] = pool_addr(a.pool, is.slot, a.bt_off + ((long long)j * a.d_out + (long long)nv0 * 8) * 2, &room);
+          sb |= (j < is.r) && (wb[h] == nullptr || room < wlen_b);
+        }
+      }
+    }
+    is.split_a = __any_sync(0xffffffffu, sa);
+    is.split_b = __any_sync(0xffffffffu, sb);
+    is.wa0 = (unsigned long long)wa[0];
+    is.wa1 = (unsigned long long)wa[1];
+    is.wb0 = (unsigned long long)wb[0];
+    is.wb1 = (unsigned long long)wb[1];
+    is.xrow = a.x ? (unsigned long long)(a.x + (long long)my_row * a.ldx + (long long)kv0 * 8) : 0ull;
+    is.yrow = a.y ? (unsigned long long)(a.y + (long long)my_row * a.ldy + (long long)nv0 * 8) : 0ull;
+    ItemInfo &I = my_info[li % kItemSlots];
+    if (lane < is.m) I.rows[lane] = my_row;
+    if (lane == 0) {
+      I.m = is.m;
+      I.r = is.r;
+      I.scale = scale;
+    }
     __syncwarp();
-    for (int idx = lane; idx < rows; idx += 32) {
-      if (idx < r) {
-        const long long off = shrink ? a.a_off + ((long long)idx * a.d_in + (long long)v_lo * 8) * 2
-                                     : a.bt_off + ((long long)idx * a.d_out + (long long)v_lo * 8) * 2;
-        copy_pool_row(a.pool, slot, off, row_bytes, buf + idx * kTileRowBytes, &full[stage], a.status);
-      } else {
-        const int i = idx - r;
-        const long long row = a.perm[pbeg + i];
-        const uint16_t *src = shrink ? a.x + row * a.ldx + (long long)v_lo * 8
-                                     : a.y + row * a.ldy + (long long)v_lo * 8;
-        bulk_g2s(buf + act_base + i * kTileRowBytes, src, row_bytes, &full[stage]);
-      }
-    }
   };
 
-  if (warp == 0) {
-    for (long long g = 0; g < total_tiles && g < kStages; ++g) issue(g);
-  }
-
-  auto exchange = [&](int m, int r) {
-    cluster.sync();  // every CTA's partial sums are complete
-    for (int idx = tid; idx < m * r; idx += kDecodeThreads) {
-      const int i = idx / r, j = idx - (idx / r) * r;
-      float sum = 0.f;
-      for (int c = 0; c < C; ++c) sum += cluster.map_shared_rank(s_part, c)[i * kRMax + j];
-      s_v[i * kRMax + j] = sum;
-    }
-    cluster.sync();  // peers are done reading this CTA's partials
-  };
-
-  long long g = 0;
-  for (int li = 0; li < my_items; ++li) {
-    const int4 d = a.items[cid + li * ncl];
-    const int slot = d.x, pbeg = d.y, m = d.z;
-    const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
-    const float scale = a.scales[slot];
-    __syncthreads();  // the previous item no longer uses s_rows / s_part / s_v
-    if (tid < m) s_rows[tid] = a.perm[pbeg + tid];
-    if (MODE != kExpandOnly) {
-      for (int idx = tid; idx < kItemRows * kRMax; idx += kDecodeThreads) s_part[idx] = 0.f;
-    } else {
-      for (int idx = tid; idx < m * r; idx += kDecodeThreads) {
-        const int i = idx / r, j = idx - (idx / r) * r;
-        s_v[i * kRMax + j] = a.v[(long long)a.perm[pbeg + i] * a.ldv + j];
-      }
-    }
-    __syncthreads();
-    const int jb = r <= 8 ? 1 : r <= 16 ? 2 : r <= 32 ? 4 : 8;
-    for (int tt = 0; tt < tpi; ++tt, ++g) {
-      if (MODE == kFused && tt == nk && r > 0 && m > 0) exchange(m, r);
-      const int stage = (int)(g % kStages);
-      const uint32_t parity = (uint32_t)((g / kStages) & 1);
-      const bool ok = mbar_wait_bounded(&full[stage], parity, a.status);
-      if (ok && r > 0 && m > 0) {
-        const uint8_t *buf = ring + stage * a.stage_bytes;
-        const bool shrink = tt < nk;
-        const int t_idx = shrink ? tt : tt - nk;
-        const int v_lo = (shrink ? kv0 : nv0) + t_idx * kTileVecs;
-        const int wv = max(0, min(v_lo + kTileVecs, shrink ? kv1 : nv1) - v_lo);
-        if (wv > 0) {
-          if (shrink) {
-            switch (jb) {
-              case 1: shrink_tile<1>(buf, act_base, wv, r, m, s_part, lane, warp); break;
-              case 2: shrink_tile<2>(buf, act_base, wv, r, m, s_part, lane, warp); break;
-              case 4: shrink_tile<4>(buf, act_base, wv, r, m, s_part, lane, warp); break;
-              default: shrink_tile<8>(buf, act_base, wv, r, m, s_part, lane, warp); break;
+  // ---- copy this warp's share of the next tile into `stage`: tile row q
+  // (weight rows first, then activation rows) is copied by warp q % 8, one
+  // 16-byte cp.async per lane, so a row is one coalesced warp instruction.
+  auto issue_next = [&](int stage) {
+    if (is.tt == 0) resolve(is.li);
+    const bool shrink = is.tt < nk;
+    const int t_idx = shrink ? is.tt : is.tt - nk;
+    const int v_lo = (shrink ? kv0 : nv0) + t_idx * TV;
+    const int wv = max(0, min(v_lo + TV, shrink ? kv1 : nv1) - v_lo);
+    const int rows = (wv > 0 && is.r > 0 && is.m > 0) ? is.r + is.m : 0;
+    uint8_t *buf = S.ring + stage * a.stage_bytes;
+    const bool on0 = lane < wv, on1 = lane + 32 < wv;
+    const unsigned long long w0 = shrink ? is.wa0 : is.wb0, w1 = shrink ? is.wa1 : is.wb1;
+    const bool split = shrink ? is.split_a : is.split_b;
+    const unsigned long long act = shrink ? is.xrow : is.yrow;
+    for (int q = warp; q < rows; q += kConsumerWarps) {
+      if (q < is.r) {
+        const unsigned long long base = __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h == 0 ? !on0 : !on1) continue;
+          const int vec = lane + 32 * h;
+          const uint8_t *src = reinterpret_cast<const uint8_t *>(base) + (long long)t_idx * TV * 16 + vec * 16;
+          if (split) {  // the slice crosses a page: translate this chunk on its own
+            long long room;
+            const long long off = (shrink ? a.a_off + (long long)q * a.d_in * 2 : a.bt_off + (long long)q * a.d_out * 2) +
+                                  (long long)(v_lo + vec) * 16;
+            src = pool_addr(a.pool, is.slot, off, &room);
+            if (src == nullptr) {
+              set_status(a.status, LORA_ERR_NOT_LOADED);
+              src = a.pool.base;
             }
-          } else {
-            expand_tile(buf, act_base, wv, v_lo, r, m, s_v, scale, s_rows, a, lane, warp);
           }
+          cp_async16(buf + q * pitch + vec * 16, src);
         }
+      } else {
+        const int i = q - is.r;
+        const unsigned long long base = __shfl_sync(0xffffffffu, act, i);
+        const uint16_t *src = reinterpret_cast<const uint16_t *>(base) + (long long)t_idx * TV * 8;
+        if (on0) cp_async16(buf + act_base + i * pitch + lane * 16, src + lane * 8);
+        if (on1) cp_async16(buf + act_base + i * pitch + (lane + 32) * 16, src + (lane + 32) * 8);
       }
-      __syncthreads();  // stage consumed by every thread
-      if (warp == 0 && g + kStages < total_tiles) issue(g + kStages);
     }
-    if (MODE == kShrinkOnly && r > 0 && m > 0) {
-      exchange(m, r);
+    cp_async_arrive(&S.full[stage]);
+    if (++is.tt == tpi) {
+      is.tt = 0;
+      ++is.li;
+    }
+  };
+
+  // prologue: fill the ring
+  for (int k = 0; k < total && k < NS; ++k) issue_next(k);
+
+  bool joined = false;  // start barrier completed (needed before the first push)
+  int xi = 0;           // exchange counter
+  int c_stage = 0;
+  uint32_t c_phase = 0;
+  int li = 0, tt = 0, m = 0, r = 0;
+  float scale = 0.f;
+  float sacc[ShrinkShape<JB>::NACC];  // this lane's dot products of the item so far
+  for (int g = 0; g < total; ++g) {
+    const int stage = c_stage;
+    const uint32_t phase = c_phase;
+    if (++c_stage == NS) {
+      c_stage = 0;
+      c_phase ^= 1u;
+    }
+    const ItemInfo &I = my_info[li % kItemSlots];
+    if (tt == 0) {
+      m = I.m;
+      r = I.r;
+      scale = I.scale;
+#pragma unroll
+      for (int k = 0; k < ShrinkShape<JB>::NACC; ++k) sacc[k] = 0.f;
+    }
+    const bool live = r > 0 && m > 0;
+    if (MODE == kFused && tt == nk && live) {
+      // this CTA's split-K share of v is complete: push it to every CTA of
+      // the cluster (itself included), then sum what arrived, in fixed CTA
+      // order
+      shrink_spill<JB>(sacc, r, m, S.red + warp * recv_slice, lane);
+      __syncthreads();
+      if (!joined) {
+        cluster_wait();
+        joined = true;
+      }
+      const int buf = xi & 1, n = m * r;
+      float *recv = S.recv + buf * C * recv_slice;
+      if (tid == 0) mbar_arrive_expect_tx(&S.recv_full[buf], (uint32_t)(C * n * 4));
+      const uint32_t recv_u = smem_u32(recv + crank * n), bar_u = smem_u32(&S.recv_full[buf]);
+      for (int e = tid; e < n; e += kConsumerThreads) {
+        float part = 0.f;  // this CTA's share of v[e], summed over the warps in fixed order
+        for (int w = 0; w < kConsumerWarps; ++w) part += S.red[w * recv_slice + e];
+        for (int c = 0; c < C; ++c) st_async_f32(mapa_u32(recv_u + 4u * e, c), part, mapa_u32(bar_u, c));
+      }
+      mbar_wait_cluster_bounded(&S.recv_full[buf], (xi >> 1) & 1, a.status);
+      for (int e = tid; e < n; e += kConsumerThreads) {
+        float sum = 0.f;
+        for (int c = 0; c < C; ++c) sum += recv[c * n + e];
+        const int i = e / r, j = e - i * r;
+        S.v[i * kRMax + j] = sum;
+      }
+      __syncthreads();
+      ++xi;
+    }
+    const bool ok = mbar_wait_bounded(&S.full[stage], phase, a.status);
+    if (MODE == kExpandOnly && tt == 0 && live) {
+      for (int idx = tid; idx < m * r; idx += kConsumerThreads) {
+        const int i = idx / r, j = idx - i * r;
+        S.v[i * kRMax + j] = a.v[(long long)I.rows[i] * a.ldv + j];
+      }
+      __syncthreads();
+    }
+    if (ok && live) {
+      const uint8_t *buf = S.ring + stage * a.stage_bytes;
+      const bool shrink = tt < nk;
+      const int t_idx = shrink ? tt : tt - nk;
+      const int v_lo = (shrink ? kv0 : nv0) + t_idx * TV;
+      const int wv = max(0, min(v_lo + TV, shrink ? kv1 : nv1) - v_lo);
+      if (shrink) {
+        shrink_accumulate<JB>(buf, act_base, pitch, wv, r, m, sacc, lane, warp);
+      } else if (wv > 0) {
+        expand_tile(buf, act_base, pitch, wv, v_lo, r, m, S.v, scale, I.rows, a, tid);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.empty[stage]);  // this warp is done with the stage
+    if (g + NS < total) {                          // refill it once every warp is
+      mbar_wait_bounded(&S.empty[stage], phase, a.status);
+      issue_next(stage);
+    }
+    if (MODE == kShrinkOnly && tt == tpi - 1 && live) {
+      shrink_spill<JB>(sacc, r, m, S.red + warp * recv_slice, lane);
+      __syncthreads();
+      if (!joined) {
+        cluster_wait();
+        joined = true;
+      }
+      const int buf = xi & 1, n = m * r;
+      float *recv = S.recv + buf * C * recv_slice;
+      if (tid == 0) mbar_arrive_expect_tx(&S.recv_full[buf], (uint32_t)(C * n * 4));
+      const uint32_t recv_u = smem_u32(recv + crank * n), bar_u = smem_u32(&S.recv_full[buf]);
+      for (int e = tid; e < n; e += kConsumerThreads) {
+        float part = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) part += S.red[w * recv_slice + e];
+        for (int c = 0; c < C; ++c) st_async_f32(mapa_u32(recv_u + 4u * e, c), part, mapa_u32(bar_u, c));
+      }
+      mbar_wait_cluster_bounded(&S.recv_full[buf], (xi >> 1) & 1, a.status);
       if (crank == 0) {
-        for (int idx = tid; idx < m * a.r_max; idx += kDecodeThreads) {
-          const int i = idx / a.r_max, j = idx - (idx / a.r_max) * a.r_max;
-          a.v[(long long)s_rows[i] * a.ldv + j] = j < r ? s_v[i * kRMax + j] : 0.f;
+        for (int idx = tid; idx < m * a.r_max; idx += kConsumerThreads) {
+          const int i = idx / a.r_max, j = idx - i * a.r_max;
+          float sum = 0.f;
+          if (j < r)
+            for (int c = 0; c < C; ++c) sum += recv[c * n + i * r + j];
+          a.v[(long long)I.rows[i] * a.ldv + j] = sum;
         }
       }
+      __syncthreads();
+      ++xi;
+    }
+    if (++tt == tpi) {
+      tt = 0;
+      ++li;
     }
   }
+  if (!joined) cluster_wait();
+  // No CTA leaves while a peer may still write into its shared memory.
+  cluster_arrive();
+  cluster_wait();
   griddep_launch_dependents();
 }
 
-static int decode_smem_bytes(int r_max, int *stage_bytes) {
-  *stage_bytes = (r_max + kItemRows) * kTileRowBytes;
-  return kStages * *stage_bytes + kStages * 8 + 2 * kItemRows * kRMax * 4 + kItemRows * 4;
+// Ring geometry for a slot rank: 1 KiB rows and two stages (one shrink and one
+// expand tile of a d=4096 item in flight) up to rank 32; 512-byte rows beyond.
+static void decode_geometry(int r_max, int *tile_vecs, int *row_pitch, int *n_stages) {
+  *tile_vecs = r_max <= 32 ? 64 : 32;
+  *row_pitch = *tile_vecs * 16 + 16;
+  *n_stages = 2;
 }
 
-template <int MODE>
-static cudaError_t launch_mode(const DecodeArgs &a, int n_clusters, int smem, cudaStream_t st) {
+static int decode_smem_bytes(int r_max, int *stage_bytes, int *n_stages) {
+  int tv, pitch;
+  decode_geometry(r_max, &tv, &pitch, n_stages);
+  *stage_bytes = (r_max + kItemRows) * pitch;
+  return *n_stages * *stage_bytes + (2 * kMaxStages + 2) * 8 + kConsumerWarps * kItemSlots * (int)sizeof(ItemInfo) +
+         kConsumerWarps * kItemRows * r_max * 4 + kItemRows * kRMax * 4 + 2 * kClusterCtas * kItemRows * r_max * 4;
+}
+
+// Rank rows per warp of the shrink: the smallest power of two with
+// 8 * JB >= r_max (ranks below r_max use the same kernel).
+static int jb_for(int r_max) { return r_max <= 8 ? 1 : r_max <= 16 ? 2 : r_max <= 32 ? 4 : 8; }
+
+template <int MODE, int JB>
+static cudaError_t launch_one(const DecodeArgs &a, int n_clusters, int smem, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_clusters * kClusterCtas);
   cfg.blockDim = dim3(kDecodeThreads);
@@ -344,22 +625,47 @@ static cudaError_t launch_mode(const DecodeArgs &a, int n_clusters, int smem, cu
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<MODE>, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<MODE, JB>, a);
+}
+
+template <int MODE>
+static cudaError_t launch_mode(const DecodeArgs &a, int jb, int n_clusters, int smem, cudaStream_t st) {
+  switch (jb) {
+    case 1: return launch_one<MODE, 1>(a, n_clusters, smem, st);
+    case 2: return launch_one<MODE, 2>(a, n_clusters, smem, st);
+    case 4: return launch_one<MODE, 4>(a, n_clusters, smem, st);
+    default: return launch_one<MODE, 8>(a, n_clusters, smem, st);
+  }
+}
+
+template <int MODE, int JB>
+static cudaError_t set_smem(int bytes) {
+  return cudaFuncSetAttribute(decode_kernel<MODE, JB>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int MODE>
+static cudaError_t set_smem_all(int bytes) {
+  cudaError_t e = set_smem<MODE, 1>(bytes);
+  if (e == cudaSuccess) e = set_smem<MODE, 2>(bytes);
+  if (e == cudaSuccess) e = set_smem<MODE, 4>(bytes);
+  if (e == cudaSuccess) e = set_smem<MODE, 8>(bytes);
+  return e;
+}
+
+template <int JB>
+static cudaError_t max_clusters(int *n, const cudaLaunchConfig_t *cfg) {
+  return cudaOccupancyMaxActiveClusters(n, decode_kernel<kFused, JB>, cfg);
 }
 
 int decode_setup(lora_pool *pool) {
-  int stage;
-  const int smem = decode_smem_bytes(pool->r_max, &stage);
+  int stage, ns;
+  const int smem = decode_smem_bytes(pool->r_max, &stage, &ns);
   pool->decode_smem = smem;
   // The attribute is per function: set it to what the largest rank needs, so
   // that pools of different r_max can coexist.
-  const int smem_cap = decode_smem_bytes(kRMax, &stage);
-  if (cudaFuncSetAttribute(decode_kernel<kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(decode_kernel<kShrinkOnly>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(decode_kernel<kExpandOnly>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_cap) !=
-          cudaSuccess)
+  const int smem_cap = decode_smem_bytes(kRMax, &stage, &ns);
+  if (set_smem_all<kFused>(smem_cap) != cudaSuccess || set_smem_all<kShrinkOnly>(smem_cap) != cudaSuccess ||
+      set_smem_all<kExpandOnly>(smem_cap) != cudaSuccess)
     return LORA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kClusterCtas);
@@ -373,7 +679,14 @@ int decode_setup(lora_pool *pool) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<kFused>, &cfg) != cudaSuccess || n < 1) return LORA_ERR_CUDA;
+  cudaError_t e;
+  switch (jb_for(pool->r_max)) {
+    case 1: e = max_clusters<1>(&n, &cfg); break;
+    case 2: e = max_clusters<2>(&n, &cfg); break;
+    case 4: e = max_clusters<4>(&n, &cfg); break;
+    default: e = max_clusters<8>(&n, &cfg); break;
+  }
+  if (e != cudaSuccess || n < 1) return LORA_ERR_CUDA;
   pool->decode_max_clusters = n;
   return LORA_OK;
 }
@@ -408,9 +721,11 @@ int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, in
   a.ldv = ldv;
   a.status = pool->d_status;
   a.items_hdr = items_hdr;
-  int stage;
-  const int smem = decode_smem_bytes(pool->r_max, &stage);
+  int stage, ns;
+  const int smem = decode_smem_bytes(pool->r_max, &stage, &ns);
   a.stage_bytes = stage;
+  a.n_stages = ns;
+  decode_geometry(pool->r_max, &a.tile_vecs, &a.row_pitch, &ns);
   // Items are bounded by min(T, n_slots) segments plus T / kItemRows chunk
   // splits; clusters loop over items, so the grid never exceeds what fits.
   const long long bound = (long long)std::min(T, pool->n_slots) + (T + kItemRows - 1) / kItemRows;
@@ -418,9 +733,10 @@ int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, in
   if (n_clusters < 1) n_clusters = 1;
   cudaError_t e;
   g_launches.fetch_add(1);
-  if (mode == kFused) e = launch_mode<kFused>(a, n_clusters, smem, st);
-  else if (mode == kShrinkOnly) e = launch_mode<kShrinkOnly>(a, n_clusters, smem, st);
-  else e = launch_mode<kExpandOnly>(a, n_clusters, smem, st);
+  const int jb = jb_for(pool->r_max);
+  if (mode == kFused) e = launch_mode<kFused>(a, jb, n_clusters, smem, st);
+  else if (mode == kShrinkOnly) e = launch_mode<kShrinkOnly>(a, jb, n_clusters, smem, st);
+  else e = launch_mode<kExpandOnly>(a, jb, n_clusters, smem, st);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return LORA_ERR_CUDA;
