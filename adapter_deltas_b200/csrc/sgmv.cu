@@ -28,7 +28,6 @@
 
 #include "internal.cuh"
 
-
 namespace lora {
 
 struct DecodeArgs {
@@ -73,147 +72,147 @@ __device__ __forceinline__ void copy_pool_row(const PoolView &pool, int slot, lo
   }
 }
 
-// Shrink, output-stationary.  Lane l owns rank j = l % RW of the adapter
-// (and j + 32 when the slot rank exceeds 32) and the rows i = l / RW (mod NH)
-// of the item, RW = min(8 JB, 32) lanes per row phase, NH = 32 / RW phases.
-// Warp w takes the 16-byte column vectors w, w + 8, ... of every tile, so the
-// K dimension is split over the warps (and over the cluster's CTAs), and each
-// lane accumulates complete dot products of its outputs in registers for the
-// whole item: no cross-lane reduction.  The warps' partial sums are added in
-// shared memory once per item.
+// ------------------------------------------------------------ warp MMA
+// The decode contractions are tiny (an item has at most 16 rows and the rank
+// is at most 64), so they run on warp-level mma.sync m16n8k16 (bf16 inputs,
+// fp32 accumulators in registers), fed by ldmatrix from the staged rows:
+// one instruction does 16 x 8 x 16 multiply-adds on bf16 operands as they are,
+// where the same work on the FMA pipes needs a conversion per element.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Shrink: this warp's share of V[i][j] = sum_k x[i][k] A[j][k] over the
+// tile's columns, accumulated in acc[n-tile][4] (rows g, g + 8 and columns
+// 2t, 2t + 1 of each 8-rank n-tile; g = lane / 4, t = lane % 4).  The warps
+// split the tile's 16-column k-steps.  Rows i >= m and ranks j >= r read row 0
+// of their operand instead: an output element depends only on its own row of
+// each operand, so those lanes' results are simply never spilled.  An odd
+// last vector (8 columns) zeroes both operands' upper k half.
 template <int JB>
-struct ShrinkShape {
-  static constexpr int RW = JB * 8 < 32 ? JB * 8 : 32;  // lanes sharing one row phase
-  static constexpr int NH = 32 / RW;                     // row phases
-  static constexpr int NJ = JB * 8 > 32 ? 2 : 1;         // ranks per lane
-  static constexpr int NU = kItemRows / NH;              // rows per lane
-  static constexpr int NACC = NU * NJ;
+__device__ __forceinline__ void shrink_mma(uint32_t buf_u, uint32_t act_u, int pitch, int wv, int r, int m,
+                                           float (&acc)[JB < 2 ? 2 : JB][4], int lane, int warp) {
+  constexpr int NT = JB < 2 ? 2 : JB;  // 8-rank n-tiles (loaded two at a time)
+  const int ksteps = (wv + 1) / 2;     // 16 columns = two 16-byte vectors
+  const int xr = (lane & 7) + ((lane >> 3) & 1) * 8, xk = (lane >> 4) * 16;
+  const uint32_t xrow = act_u + (xr < m ? xr : 0) * pitch + xk;
+  uint32_t arow[NT / 2];
+#pragma unroll
+  for (int p = 0; p < NT / 2; ++p) {
+    const int j = (lane & 7) + (lane >> 4) * 8 + 16 * p, ak = ((lane >> 3) & 1) * 16;
+    arow[p] = buf_u + (j < r ? j : 0) * pitch + ak;
+  }
+  for (int ks = warp; ks < ksteps; ks += kConsumerWarps) {
+    const bool half = 2 * ks + 1 >= wv;
+    uint32_t a[4];
+    ldsm_x4(xrow + ks * 32, a);
+    if (half) a[2] = a[3] = 0u;
+#pragma unroll
+    for (int p = 0; p < NT / 2; ++p) {
+      uint32_t b[4];
+      ldsm_x4(arow[p] + ks * 32, b);
+      if (half) b[1] = b[3] = 0u;
+      mma_bf16_16816(acc[2 * p], a, b[0], b[1]);
+      mma_bf16_16816(acc[2 * p + 1], a, b[2], b[3]);
+    }
+  }
+}
+
+// This warp's partial V of the item -> red[i * r + j] (rows < m, ranks < r).
+template <int JB>
+__device__ __forceinline__ void shrink_spill(const float (&acc)[JB < 2 ? 2 : JB][4], int r, int m, float *red,
+                                             int lane) {
+  constexpr int NT = JB < 2 ? 2 : JB;
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int i = g + (h >> 1) * 8, j = nt * 8 + 2 * t + (h & 1);
+      if (i < m && j < r) red[i * r + j] = acc[nt][h];
+    }
+  }
+}
+
+// Expand: y[i][n] = bf16_rn(y + scale * sum_j V[i][j] B^T[j][n]) for the
+// tile's columns.  V enters the MMA as two bf16 terms (hi + lo: about 16 bits
+// of each fp32 value), built in registers once per item; B^T rows are loaded
+// transposed by ldmatrix.  Warp w takes the 16-column groups w, w + 8, ...
+template <int JB>
+struct ExpandA {
+  static constexpr int KS = JB < 2 ? 1 : JB / 2;  // 16-rank k-steps
+  uint32_t hi[KS][4], lo[KS][4];
 };
 
 template <int JB>
-__device__ __forceinline__ void shrink_accumulate(const uint8_t *buf, int act_base, int pitch, int wv, int r, int m,
-                                                  float (&acc)[ShrinkShape<JB>::NACC], int lane, int warp) {
-  using SS = ShrinkShape<JB>;
-  const int jl = lane % SS::RW, ih = lane / SS::RW;
-  for (int kv = warp; kv < wv; kv += kConsumerWarps) {
-    float av[SS::NJ][8];
+__device__ __forceinline__ void expand_prepare(const float *s_v, int r, int m, ExpandA<JB> &A, int lane) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int h = 0; h < SS::NJ; ++h) {
-      const int j = jl + 32 * h;
-      if (j < r) {
-        unpack8(*reinterpret_cast<const uint4 *>(buf + j * pitch + kv * 16), av[h]);
-      } else {
+  for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) av[h][e] = 0.f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < SS::NU; ++u) {
-      const int i = ih + SS::NH * u;
-      if (i < m) {
-        float xv[8];
-        unpack8(*reinterpret_cast<const uint4 *>(buf + act_base + i * pitch + kv * 16), xv);
-#pragma unroll
-        for (int h = 0; h < SS::NJ; ++h) {
-          float s0 = acc[u * SS::NJ + h], s1 = av[h][1] * xv[1];
-          s0 = fmaf(av[h][0], xv[0], s0);
-          s1 = fmaf(av[h][3], xv[3], s1);
-          s0 = fmaf(av[h][2], xv[2], s0);
-          s1 = fmaf(av[h][5], xv[5], s1);
-          s0 = fmaf(av[h][4], xv[4], s0);
-          s1 = fmaf(av[h][7], xv[7], s1);
-          s0 = fmaf(av[h][6], xv[6], s0);
-          acc[u * SS::NJ + h] = s0 + s1;
-        }
-      }
+    for (int q = 0; q < 4; ++q) {  // a0: (g, 2t), a1: (g+8, 2t), a2: (g, 2t+8), a3: (g+8, 2t+8)
+      const int i = g + (q & 1) * 8, j = 16 * ks + 2 * t + (q >> 1) * 8;
+      const float v0 = (i < m && j < r) ? s_v[i * kRMax + j] : 0.f;
+      const float v1 = (i < m && j + 1 < r) ? s_v[i * kRMax + j + 1] : 0.f;
+      const uint32_t h = pack_bf16x2(v0, v1);
+      A.hi[ks][q] = h;
+      A.lo[ks][q] = pack_bf16x2(v0 - bf16_lo(h), v1 - bf16_hi(h));
     }
   }
 }
 
-// This warp's partial sums of the item -> red[warp][i * r + j].
 template <int JB>
-__device__ __forceinline__ void shrink_spill(const float (&acc)[ShrinkShape<JB>::NACC], int r, int m, float *red,
-                                             int lane) {
-  using SS = ShrinkShape<JB>;
-  const int jl = lane % SS::RW, ih = lane / SS::RW;
+__device__ __forceinline__ void expand_mma(uint32_t buf_u, const uint8_t *yb, uint32_t zero_u, int pitch, int wv,
+                                           int v_lo, int r, int m, const ExpandA<JB> &A, float scale,
+                                           const int *s_rows, const DecodeArgs &a, int lane, int warp) {
+  const int g = lane >> 2, t = lane & 3;
+  const int groups = (wv + 1) / 2;  // 16-column groups (an odd last vector is half a group)
+  const int bj = (lane & 7) + ((lane >> 3) & 1) * 8, bn = (lane >> 4) * 16;
+  for (int cg = warp; cg < groups; cg += kConsumerWarps) {
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-  for (int u = 0; u < SS::NU; ++u) {
-    const int i = ih + SS::NH * u;
-#pragma unroll
-    for (int h = 0; h < SS::NJ; ++h) {
-      const int j = jl + 32 * h;
-      if (i < m && j < r) red[i * r + j] = acc[u * SS::NJ + h];
+    for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
+      // ranks j >= r read 16 zero bytes: their V is zero and stale weights
+      // (possibly not finite) must not meet it
+      const int j = 16 * ks + bj;
+      uint32_t b[4];
+      ldsm_x4_t(j < r ? buf_u + j * pitch + cg * 32 + bn : zero_u + bn, b);
+      mma_bf16_16816(acc[0], A.hi[ks], b[0], b[1]);
+      mma_bf16_16816(acc[0], A.lo[ks], b[0], b[1]);
+      mma_bf16_16816(acc[1], A.hi[ks], b[2], b[3]);
+      mma_bf16_16816(acc[1], A.lo[ks], b[2], b[3]);
     }
-  }
-}
-
-// One expand tile: columns [v_lo*8, v_lo*8 + wv*8) of d_out.  Work units are
-// (group of RT rows, 4 consecutive columns), spread over all threads of the
-// CTA; a unit walks the ranks 4 at a time (loads first, then FMAs), so every
-// B vector it loads serves its RT rows.  RT = 4 for items of more than four
-// rows, else 1.
-template <int RT>
-__device__ __forceinline__ void expand_units(const uint8_t *buf, int act_base, int pitch, int wv, int v_lo, int r, int m,
-                                             const float *s_v, float scale, const int *s_rows, const DecodeArgs &a,
-                                             int tid) {
-  const int n4 = 2 * wv;                 // 4-column units per row
-  const int groups = (m + RT - 1) / RT;
-  for (int idx = tid; idx < groups * n4; idx += kConsumerThreads) {
-    const int gi = idx / n4, c4 = idx - gi * n4;
-    float acc[RT][4];
+    const int n_nt = 2 * cg + 1 < wv ? 2 : 1;
 #pragma unroll
-    for (int k = 0; k < RT; ++k)
+    for (int nt = 0; nt < 2; ++nt) {
+      if (nt >= n_nt) break;
+      const int col = cg * 16 + nt * 8 + 2 * t;  // within the tile
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
-    const uint8_t *bcol = buf + c4 * 8;
-    for (int j0 = 0; j0 < r; j0 += 4) {
-      float b[4][4], c[RT][4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = j0 + u;
-        if (j < r) {
-          const uint2 q = *reinterpret_cast<const uint2 *>(bcol + j * pitch);
-          b[u][0] = bf16_lo(q.x);
-          b[u][1] = bf16_hi(q.x);
-          b[u][2] = bf16_lo(q.y);
-          b[u][3] = bf16_hi(q.y);
-#pragma unroll
-          for (int k = 0; k < RT; ++k) c[k][u] = s_v[(gi * RT + k) * kRMax + j];
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) b[u][e] = 0.f;
-#pragma unroll
-          for (int k = 0; k < RT; ++k) c[k][u] = 0.f;
+      for (int hr = 0; hr < 2; ++hr) {
+        const int i = g + hr * 8;
+        if (i < m) {
+          const uint32_t yv = *reinterpret_cast<const uint32_t *>(yb + i * pitch + col * 2);
+          const uint32_t o = pack_bf16x2(fmaf(scale, acc[nt][2 * hr], bf16_lo(yv)),
+                                         fmaf(scale, acc[nt][2 * hr + 1], bf16_hi(yv)));
+          *reinterpret_cast<uint32_t *>(a.y + (long long)s_rows[i] * a.ldy + (long long)v_lo * 8 + col) = o;
         }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int k = 0; k < RT; ++k)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[k][e] = fmaf(c[k][u], b[u][e], acc[k][e]);
-    }
-#pragma unroll
-    for (int k = 0; k < RT; ++k) {
-      const int i = gi * RT + k;
-      if (i < m) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(buf + act_base + i * pitch + c4 * 8);
-        uint2 o;
-        o.x = pack_bf16x2(fmaf(scale, acc[k][0], bf16_lo(u.x)), fmaf(scale, acc[k][1], bf16_hi(u.x)));
-        o.y = pack_bf16x2(fmaf(scale, acc[k][2], bf16_lo(u.y)), fmaf(scale, acc[k][3], bf16_hi(u.y)));
-        *reinterpret_cast<uint2 *>(a.y + (long long)s_rows[i] * a.ldy + (long long)v_lo * 8 + c4 * 4) = o;
-      }
     }
   }
-}
-
-__device__ __forceinline__ void expand_tile(const uint8_t *buf, int act_base, int pitch, int wv, int v_lo, int r,
-                                            int m, const float *s_v, float scale, const int *s_rows,
-                                            const DecodeArgs &a, int tid) {
-  if (m <= 4)
-    expand_units<1>(buf, act_base, pitch, wv, v_lo, r, m, s_v, scale, s_rows, a, tid);
-  else
-    expand_units<4>(buf, act_base, pitch, wv, v_lo, r, m, s_v, scale, s_rows, a, tid);
 }
 
 // ------------------------------------------------------------ cluster helpers
@@ -294,6 +293,7 @@ struct ItemInfo {
 struct DecodeSmem {
   uint8_t *ring;
   uint64_t *full, *empty, *recv_full;
+  uint8_t *zero;   // 32 zero bytes: the expand's operand rows beyond the rank
   ItemInfo *info;  // [kConsumerWarps][kItemSlots]
   float *red;      // [kConsumerWarps][kItemRows * r_max]: the warps' shrink partials
   float *v, *recv;
@@ -306,6 +306,7 @@ __device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeAr
   S.full = reinterpret_cast<uint64_t *>(p); p += kMaxStages * 8;
   S.empty = reinterpret_cast<uint64_t *>(p); p += kMaxStages * 8;
   S.recv_full = reinterpret_cast<uint64_t *>(p); p += 2 * 8;
+  S.zero = p; p += 32;
   S.info = reinterpret_cast<ItemInfo *>(p); p += kConsumerWarps * kItemSlots * sizeof(ItemInfo);
   S.red = reinterpret_cast<float *>(p); p += kConsumerWarps * kItemRows * a.r_max * 4;
   S.v = reinterpret_cast<float *>(p); p += kItemRows * kRMax * 4;
@@ -325,7 +326,7 @@ struct IssueState {
 };
 
 template <int MODE, int JB>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel(const DecodeArgs a) {
   const int C = (int)cluster_nctarank();
   const int crank = (int)cluster_ctarank();
   const int cid = blockIdx.x / C, ncl = gridDim.x / C;
@@ -348,6 +349,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
     mbar_init(&S.recv_full[1], 1);
     fence_mbar_init();
   }
+  if (tid < 8) reinterpret_cast<uint32_t *>(S.zero)[tid] = 0u;
   __syncthreads();
   // Peers may push into this CTA's shared memory only after its barriers are
   // initialised: arrive now, wait before the first push.
@@ -478,7 +480,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
   uint32_t c_phase = 0;
   int li = 0, tt = 0, m = 0, r = 0;
   float scale = 0.f;
-  float sacc[ShrinkShape<JB>::NACC];  // this lane's dot products of the item so far
+  float sacc[JB < 2 ? 2 : JB][4];  // this warp's MMA fragment of the item's V so far
+  ExpandA<JB> va;                  // the item's V as MMA operand fragments (hi + lo)
   for (int g = 0; g < total; ++g) {
     const int stage = c_stage;
     const uint32_t phase = c_phase;
@@ -492,7 +495,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
       r = I.r;
       scale = I.scale;
 #pragma unroll
-      for (int k = 0; k < ShrinkShape<JB>::NACC; ++k) sacc[k] = 0.f;
+      for (int nt = 0; nt < (JB < 2 ? 2 : JB); ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
     }
     const bool live = r > 0 && m > 0;
     if (MODE == kFused && tt == nk && live) {
@@ -538,10 +541,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
       const int t_idx = shrink ? tt : tt - nk;
       const int v_lo = (shrink ? kv0 : nv0) + t_idx * TV;
       const int wv = max(0, min(v_lo + TV, shrink ? kv1 : nv1) - v_lo);
+      const uint32_t buf_u = smem_u32(buf);
       if (shrink) {
-        shrink_accumulate<JB>(buf, act_base, pitch, wv, r, m, sacc, lane, warp);
-      } else if (wv > 0) {
-        expand_tile(buf, act_base, pitch, wv, v_lo, r, m, S.v, scale, I.rows, a, tid);
+        shrink_mma<JB>(buf_u, buf_u + act_base, pitch, wv, r, m, sacc, lane, warp);
+      } else {
+        if (t_idx == 0) expand_prepare<JB>(S.v, r, m, va, lane);
+        if (wv > 0)
+          expand_mma<JB>(buf_u, buf + act_base, smem_u32(S.zero), pitch, wv, v_lo, r, m, va, scale, I.rows, a, lane,
+                         warp);
       }
     }
     __syncwarp();
@@ -603,7 +610,7 @@ static int decode_smem_bytes(int r_max, int *stage_bytes, int *n_stages) {
   int tv, pitch;
   decode_geometry(r_max, &tv, &pitch, n_stages);
   *stage_bytes = (r_max + kItemRows) * pitch;
-  return *n_stages * *stage_bytes + (2 * kMaxStages + 2) * 8 + kConsumerWarps * kItemSlots * (int)sizeof(ItemInfo) +
+  return *n_stages * *stage_bytes + (2 * kMaxStages + 2) * 8 + 32 + kConsumerWarps * kItemSlots * (int)sizeof(ItemInfo) +
          kConsumerWarps * kItemRows * r_max * 4 + kItemRows * kRMax * 4 + 2 * kClusterCtas * kItemRows * r_max * 4;
 }
 
