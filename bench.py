@@ -66,10 +66,10 @@ def algorithmic_bytes(w, target: int, ids) -> int:
     return adapters + act.size * d_in * 2 + act.size * d_out * 4
 
 
-def traffic_from_profile(kernel_file: str, workload: str):
+def traffic_from_profile(kernel: str, kernel_file: str, workload: str):
     """DRAM bytes per launch recorded from an ncu capture, if it was taken on
     the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "decode_kernel_%s.txt" % workload)
+    path = os.path.join(ROOT, "profiles", "%s_%s.txt" % (kernel, workload))
     try:
         lines = open(path).read().splitlines()
     except OSError:
@@ -225,6 +225,10 @@ def run_b200(args, rank: int, world: int, local_rank: int):
             adapters[s] = (bf16(A), bf16(B))
     x0, y0 = bf16(w.x(target)), bf16(w.y_in(target))
     ids0 = torch.from_numpy(w.ids).to(dev)
+    # the prefill workload enters through its segment offsets (the tensor-core path)
+    segmented = args.workload == "prefill"
+    off0 = torch.from_numpy(w.seg_offsets).to(dev) if segmented else None
+    sl0 = torch.from_numpy(w.seg_slot).to(dev) if segmented else None
     sets = []
     for k in range(n_sets):
         mem = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
@@ -232,12 +236,18 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         for s, (A, B) in adapters.items():
             L.lora_pool_load(pool, s, target, int(w.rank[s]), A, B)
         ws = torch.zeros(L.lora_workspace_bytes(pool, target, w.T), dtype=torch.uint8, device=dev)
-        sets.append(dict(pool=pool, x=x0.clone(), y=y0.clone(), ids=ids0.clone(), ws=ws))
+        sets.append(dict(pool=pool, x=x0.clone(), y=y0.clone(), ids=ids0.clone(), ws=ws,
+                         off=off0.clone() if segmented else None, sl=sl0.clone() if segmented else None))
     torch.cuda.synchronize()
 
+    def call(s):
+        if segmented:
+            L.lora_apply_segments(s["pool"], target, s["x"], s["y"], s["off"], s["sl"], scales, s["ws"])
+        else:
+            L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"])
+
     def step(k):
-        s = sets[k % n_sets]
-        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"])
+        call(sets[k % n_sets])
 
     def barrier():
         if world > 1:
@@ -262,9 +272,12 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     ms = ev0.elapsed_time(ev1) / args.steps
     ms = reduce_max(ms, world, dev)
 
-    # ---- dominant kernel alone: the fused shrink/expand launch on prebuilt plans
+    # ---- dominant kernel alone: the delta launches on prebuilt plans
     for s in sets:
-        L.lora_plan_ids(s["pool"], s["ids"], s["ws"])
+        if segmented:
+            L.lora_plan_segments(s["pool"], s["off"], s["sl"], w.T, s["ws"])
+        else:
+            L.lora_plan_ids(s["pool"], s["ids"], s["ws"])
     reps = max(args.steps, 3 * n_sets)
 
     def apply_only(k):
@@ -284,7 +297,7 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     # ---- end to end through the C ABI with pinned host buffers
     xh = x0.cpu().pin_memory()
     yh = y0.cpu().pin_memory()
-    idh = ids0.cpu().pin_memory()
+    idh = (torch.cat([off0, sl0]) if segmented else ids0).cpu().pin_memory()
     yout = torch.empty_like(yh).pin_memory()
     h2d = xh.numel() * 2 + yh.numel() * 2 + idh.numel() * 4
     d2h = yout.numel() * 2
@@ -293,8 +306,13 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         s = sets[k % n_sets]
         s["x"].copy_(xh, non_blocking=True)
         s["y"].copy_(yh, non_blocking=True)
-        s["ids"].copy_(idh, non_blocking=True)
-        L.lora_apply(s["pool"], target, s["x"], s["y"], s["ids"], scales, s["ws"])
+        if segmented:
+            n_off = s["off"].numel()
+            s["off"].copy_(idh[:n_off], non_blocking=True)
+            s["sl"].copy_(idh[n_off:], non_blocking=True)
+        else:
+            s["ids"].copy_(idh, non_blocking=True)
+        call(s)
         yout.copy_(s["y"], non_blocking=True)
 
     g_ew, _ = capture_graph(dev, e2e_step, range(args.warmup))
@@ -318,6 +336,11 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     alg = algorithmic_bytes(w, target, w.ids)
     achieved = alg / (kernel_ms * 1e-3) / 1e9
     tokens = w.T * world
+    if segmented:
+        kernel_name = "prefill_kernel"
+        kernel_desc = "prefill_kernel (tcgen05) + decode_kernel launch for segments under %d rows" % L.lora_mma_min_rows()
+    else:
+        kernel_name, kernel_desc = "decode_kernel", "decode_kernel<fused>"
     line = {
         "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -330,8 +353,9 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         "hbm_gbs_step": alg * world / (ms * 1e-3) / 1e9 / world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": traffic_from_profile("sgmv.cu", args.workload),
-                     "kernel": "decode_kernel<fused>", "kernel_us": kernel_ms * 1e3,
+                     "traffic": traffic_from_profile(kernel_name, "prefill.cu" if segmented else "sgmv.cu",
+                                                     args.workload),
+                     "kernel": kernel_desc, "kernel_us": kernel_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg, "frac_of_8TBps_datasheet": achieved / 8000.0},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -339,6 +363,13 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         "clocks": clocks,
         "delta_vs_base_w_read": (kernel_ms * 1e-3) / (sum(a * b for a, b in w.targets[:1]) * 2 / (peak * 1e9)),
     }
+    if segmented:
+        # the contraction's own rate, for context: 2 flops per multiply-add of
+        # the shrink (r x d_in per row) and the expand (d_out x r per row)
+        d_in, d_out = w.targets[target]
+        rows = w.ids >= 0
+        flops = float(sum(2.0 * int(w.rank[w.ids[t]]) * (d_in + d_out) for t in np.nonzero(rows)[0]))
+        line["tensor_tflops"] = flops / (kernel_ms * 1e-3) / 1e12
     if world == 1:
         threads = min(cpu_threads(), w.T)
         v, n, el = time_oracle(w, target, args.cpu_seconds, threads)
@@ -421,7 +452,7 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
                    "deltas_per_step": n_t, "l2": "pool 31.25 GiB and 1 GiB of activations per step > L2",
                    "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": traffic_from_profile("sgmv.cu", "paged"),
+                     "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "sgmv.cu", "paged"),
                      "kernel": "decode_kernel<fused>", "kernel_us": kernel_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg},
         "gpu_launches": launches, "clocks": clocks,
