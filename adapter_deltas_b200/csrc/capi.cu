@@ -111,7 +111,7 @@ int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, i
   if (kind == kPlanIds)  // index-vector plans hold decode items only
     return launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItems);
   PrefillGeometry geo;
-  if (kind == kPlanSegments && prefill_geometry(p, target, &geo)) {
+  if (kind == kPlanSegments && prefill_geometry(p, target, plan_layout(T).j_max, &geo)) {
     // short segments on the decode kernel, long ones on the tensor cores
     rc = launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItems);
     if (rc != LORA_OK) return rc;

@@ -10,6 +10,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <unordered_map>
 #include <vector>
@@ -236,6 +237,7 @@ struct lora_pool {
   // 2 = segments, which may hold tensor-core tiles); kept on the host so that
   // an apply call can pick its kernels without reading the device.
   std::unordered_map<const void *, int> plan_kind;
+  std::map<std::pair<int, int>, int> prefill_fit;  // (cluster size, smem) -> co-resident clusters
   std::mutex mu;
 
   lora::PoolView view() const {
@@ -280,9 +282,9 @@ int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, in
                         const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
                         int items_hdr);
 struct PrefillGeometry {
-  int C, nsx, nsy, r_cap, ks_cols, ns_cols, smem;
+  int C, n_stages, r_cap, ks_cols, ns_cols, smem;
 };
-bool prefill_geometry(const lora_pool *pool, int target, PrefillGeometry *g);
+bool prefill_geometry(const lora_pool *pool, int target, int max_tiles, PrefillGeometry *g);
 int launch_prefill(lora_pool *pool, int target, const void *x, int ldx, void *y, int ldy, const float *scales,
                    int T, const void *ws, cudaStream_t st);
 int decode_setup(lora_pool *pool);
