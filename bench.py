@@ -139,20 +139,25 @@ class ClockSampler:
 # ---------------------------------------------------------------- CPU arms
 
 
-def time_oracle(w, target: int, min_seconds: float, threads: int):
-    """Run the oracle on whole batches until min_seconds passed; tokens/s."""
-    import oracle
+def oracle_inputs(w, target: int):
+    """The oracle's inputs for one batch of one target (drawn once, outside
+    any timed region)."""
     slots = [int(s) for s in np.unique(w.ids[w.ids >= 0])]
-    adapters = {s: w.adapter(s, target) for s in slots}
-    x, y = w.x(target), w.y_in(target)
+    return dict(x=w.x(target), y=w.y_in(target), adapters={s: w.adapter(s, target) for s in slots})
+
+
+def time_oracle(w, inp, min_seconds: float, threads: int, max_calls: int = 1 << 30):
+    """Run the oracle on whole batches of one target until min_seconds passed
+    (or max_calls calls); returns (calls, seconds)."""
+    import oracle
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.lora_apply(x, y, w.ids, w.n_slots, adapters, w.alpha, threads=threads)
+        oracle.lora_apply(inp["x"], inp["y"], w.ids, w.n_slots, inp["adapters"], w.alpha, threads=threads)
         n += 1
         el = time.perf_counter() - t0
-        if el >= min_seconds:
+        if el >= min_seconds or n >= max_calls:
             break
-    return n * w.T / el, n, el
+    return n, el
 
 
 def cpu_threads() -> int:
@@ -163,29 +168,45 @@ def cpu_threads() -> int:
 
 
 def run_reference(args, rank: int, world: int):
-    """The oracle, timed on the host cores, on the same workload and metric."""
+    """The oracle, timed on the host cores, on the same workload and metric.
+    A step is one batch of one target; where the workload's step covers
+    several targets of one shape (the paged workload's 128 deltas), the value
+    is scaled by their count."""
     if rank != 0:
         return
     import synth
     w = synth.config(WORKLOADS[args.workload])
+    n_t = len(w.targets) if args.workload == "paged" else 1
     threads = min(cpu_threads(), w.T)
-    for _ in range(args.warmup):
-        time_oracle(w, 0, 0.0, threads)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        time_oracle(w, 0, 0.0, threads)
-    el = time.perf_counter() - t0
-    value = args.steps * w.T / el
+    inp = oracle_inputs(w, 0)
+    time_oracle(w, inp, 0.0, threads, max_calls=args.warmup)
+    n, el = time_oracle(w, inp, 0.0, threads, max_calls=args.steps)
+    per_call = el / n
+    value = w.T / (per_call * n_t)
+    sample = "%d whole batches of %d tokens on target 0" % (n, w.T)
+    if n_t > 1:
+        sample += " (1 of the %d same-shape deltas of a step; value scaled by %d)" % (n_t, n_t)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * per_call * n_t,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.T, "seq_len": 1, "parallelism": "oracle on host cores"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": "%d whole batches of %d tokens" % (args.steps, w.T)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, n_targets: int, seconds: float):
+    """The oracle on a bounded sample of the workload (rank 0, N = 1)."""
+    threads = min(cpu_threads(), w.T)
+    inp = oracle_inputs(w, 0)
+    n, el = time_oracle(w, inp, seconds, threads)
+    sample = "%d whole batches of %d tokens on target 0 (%.1f s)" % (n, w.T, el)
+    if n_targets > 1:
+        sample += ", value scaled by the %d same-shape deltas of a step" % n_targets
+    return {"value": n * w.T / el / n_targets, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": sample}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -250,8 +271,7 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         call(sets[k % n_sets])
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        sync_ranks(world)
 
     # ---- timed region: a CUDA graph of exactly K whole steps
     g_warm, _ = capture_graph(dev, step, range(args.warmup))
@@ -336,13 +356,14 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     alg = algorithmic_bytes(w, target, w.ids)
     achieved = alg / (kernel_ms * 1e-3) / 1e9
     tokens = w.T * world
+    value = job_value(w.T, world, ms)
     if segmented:
         kernel_name = "prefill_kernel"
         kernel_desc = "prefill_kernel (tcgen05) + decode_kernel launch for segments under %d rows" % L.lora_mma_min_rows()
     else:
         kernel_name, kernel_desc = "decode_kernel", "decode_kernel<fused>"
     line = {
-        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": tokens, "seq_len": 1,
@@ -357,7 +378,7 @@ def run_b200(args, rank: int, world: int, local_rank: int):
                                                      args.workload),
                      "kernel": kernel_desc, "kernel_us": kernel_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg, "frac_of_8TBps_datasheet": achieved / 8000.0},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_value(w.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "clocks": clocks,
@@ -371,10 +392,7 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         flops = float(sum(2.0 * int(w.rank[w.ids[t]]) * (d_in + d_out) for t in np.nonzero(rows)[0]))
         line["tensor_tflops"] = flops / (kernel_ms * 1e-3) / 1e12
     if world == 1:
-        threads = min(cpu_threads(), w.T)
-        v, n, el = time_oracle(w, target, args.cpu_seconds, threads)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                "sample": "%d whole batches of %d tokens (%.1f s)" % (n, w.T, el)}
+        line["cpu_baseline"] = cpu_baseline(w, 1, args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
@@ -416,14 +434,17 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
     g_main, launches = capture_graph(dev, step, range(args.steps))
     g_warm.replay()
     torch.cuda.synchronize()
+    sync_ranks(world)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index)
     with sampler:
+        torch.cuda.synchronize()
         ev0.record()
         g_main.replay()
         ev1.record()
         torch.cuda.synchronize()
     clocks = sampler.stop()
+    sync_ranks(world)
     ms = reduce_max(ev0.elapsed_time(ev1) / args.steps, world, dev)
 
     # kernel alone: the 128 applies without the plan
@@ -437,7 +458,38 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
     ev1.record()
     torch.cuda.synchronize()
     kernel_ms = ev0.elapsed_time(ev1) / (args.steps * n_t)
-    del g_warm, g_main, g_k
+
+    # end to end: each step copies the ids and every matrix's x and y in from
+    # pinned host memory and every y back out (one staging buffer each,
+    # reused across the matrices)
+    xh = xs[0].cpu().pin_memory()
+    yh = ys[0].cpu().pin_memory()
+    idh = ids.cpu().pin_memory()
+    yout = torch.empty_like(yh).pin_memory()
+    h2d = idh.numel() * 4 + n_t * (xh.numel() + yh.numel()) * 2
+    d2h = n_t * yout.numel() * 2
+
+    def e2e_step(_k):
+        ids.copy_(idh, non_blocking=True)
+        L.lora_plan_ids(pool, ids, ws)
+        for t in range(n_t):
+            xs[t].copy_(xh, non_blocking=True)
+            ys[t].copy_(yh, non_blocking=True)
+            L.lora_apply_plan(pool, t, xs[t], ys[t], scales, ws)
+            yout.copy_(ys[t], non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 20))
+    g_e, _ = capture_graph(dev, e2e_step, range(e2e_steps))
+    g_e.replay()
+    torch.cuda.synchronize()
+    sync_ranks(world)
+    ev0.record()
+    g_e.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    sync_ranks(world)
+    e2e_ms = reduce_max(ev0.elapsed_time(ev1) / e2e_steps, world, dev)
+    del g_warm, g_main, g_k, g_e
     L.lora_pool_destroy(pool)
     if rank != 0:
         return
@@ -445,18 +497,23 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
     alg = algorithmic_bytes(w, 0, w.ids)
     achieved = alg / (kernel_ms * 1e-3) / 1e9
     line = {
-        "metric": METRIC, "value": T * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": job_value(T, world, ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": T * world, "seq_len": 1, "parallelism": "single",
+        "config": {"workload": w.name, "global_batch": T * world, "seq_len": 1,
+                   "parallelism": "replicas%d" % world if world > 1 else "single",
                    "deltas_per_step": n_t, "l2": "pool 31.25 GiB and 1 GiB of activations per step > L2",
                    "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "sgmv.cu", "paged"),
                      "kernel": "decode_kernel<fused>", "kernel_us": kernel_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg},
+        "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": launches, "clocks": clocks,
     }
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, n_t, args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
@@ -479,7 +536,9 @@ def capture_graph(dev, fn, ks):
     return g, L.lora_kernel_launches() - n0
 
 
-def reduce_max(x: float, world: int, dev) -> float:
+def reduce_max(x: float, world: int, dev=None) -> float:
+    """Max of a per-rank value over all ranks (the slowest rank sets the
+    step time); dev None reduces a host tensor (gloo)."""
     if world == 1:
         return x
     import torch
@@ -487,6 +546,18 @@ def reduce_max(x: float, world: int, dev) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def sync_ranks(world: int) -> None:
+    """Barrier of all ranks (no-op on one)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def job_value(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's batch, over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
 
 
 def main(argv=None):
