@@ -53,7 +53,9 @@ extern "C" {
 
 size_t lora_workspace_bytes(const lora_pool *p, int target, int max_tokens) {
   if (!p || target < 0 || target >= p->n_targets || max_tokens < 0 || max_tokens > kMaxTokens) return 0;
-  return plan_layout(max_tokens).total;
+  const size_t plan = plan_layout(max_tokens).total;
+  const size_t scratch = prefill_scratch_bytes(p, target, max_tokens);
+  return scratch ? align256(plan) + scratch : plan;
 }
 
 int lora_plan_layout_get(const lora_pool *p, int T, lora_plan_layout *out) {
@@ -115,7 +117,7 @@ int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, i
     // short segments on the decode kernel, long ones on the tensor cores
     rc = launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItems);
     if (rc != LORA_OK) return rc;
-    return launch_prefill(p, target, x, ldx, y, ldy, scales, T, ws, st);
+    return launch_prefill(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, st);
   }
   // every segment on the decode kernel
   return launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItemsAll);

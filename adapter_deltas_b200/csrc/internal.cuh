@@ -212,6 +212,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ void set_status(int *status, int code) { atomicCAS(status, 0, code); }
 
+// Launch attribute for programmatic dependent launch: the kernel may start
+// while the previous kernel on the stream is still running; it reads that
+// kernel's results only after griddep_wait().  Kernels of this library call
+// griddep_launch_dependents() once they have passed their own griddep_wait(),
+// so a kernel that starts early knows that everything before its
+// predecessor has completed.
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
+  return at;
+}
+
 }  // namespace lora
 
 // ---------------------------------------------------------------- host pool
@@ -237,7 +250,7 @@ struct lora_pool {
   // 2 = segments, which may hold tensor-core tiles); kept on the host so that
   // an apply call can pick its kernels without reading the device.
   std::unordered_map<const void *, int> plan_kind;
-  std::map<std::pair<int, int>, int> prefill_fit;  // (cluster size, smem) -> co-resident clusters
+  std::map<std::pair<int, int>, int> prefill_fit;  // (kernel, smem) -> co-resident CTAs
   std::mutex mu;
 
   lora::PoolView view() const {
@@ -282,11 +295,14 @@ int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, in
                         const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
                         int items_hdr);
 struct PrefillGeometry {
-  int C, n_stages, r_cap, ks_cols, ns_cols, smem;
+  int r_cap, kb_per, n_ks, n_stages, n_groups, smem_sh, smem_ex;
 };
 bool prefill_geometry(const lora_pool *pool, int target, int max_tiles, PrefillGeometry *g);
+// Workspace bytes the segment path needs after the plan (fp32 partial V of
+// every k-slice); 0 when the tensor-core path cannot serve the target.
+size_t prefill_scratch_bytes(const lora_pool *pool, int target, int T);
 int launch_prefill(lora_pool *pool, int target, const void *x, int ldx, void *y, int ldy, const float *scales,
-                   int T, const void *ws, cudaStream_t st);
+                   int T, const void *ws, size_t ws_bytes, cudaStream_t st);
 int decode_setup(lora_pool *pool);
 
 }  // namespace lora

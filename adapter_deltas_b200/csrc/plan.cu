@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_ids_kernel(const int32_t *_
   }
   for (int s = tid; s < n_slots; s += kPlanThreads) s_cnt[s] = 0;
   griddep_wait();
+  griddep_launch_dependents();  // the delta kernel may set up while the plan is built
   __syncthreads();
 
   // 1. histogram of valid ids
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
     s_bad_empty = 0;
   }
   griddep_wait();
+  griddep_launch_dependents();
   __syncthreads();
   // Offsets must be non-decreasing and inside [0, T] (then segments are
   // disjoint); otherwise the whole plan is empty.

@@ -355,6 +355,7 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   // initialised: arrive now, wait before the first push.
   cluster_arrive_relaxed();
   griddep_wait();
+  griddep_launch_dependents();
 
   // the header and this cluster's first item are read together (the items
   // array always has room for cid, whatever the count)
@@ -595,7 +596,6 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   // No CTA leaves while a peer may still write into its shared memory.
   cluster_arrive();
   cluster_wait();
-  griddep_launch_dependents();
 }
 
 // Ring geometry for a slot rank: 1 KiB rows and two stages (one shrink and one
@@ -625,13 +625,14 @@ static cudaError_t launch_one(const DecodeArgs &a, int n_clusters, int smem, cud
   cfg.blockDim = dim3(kDecodeThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kClusterCtas;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode_kernel<MODE, JB>, a);
 }
 

@@ -174,9 +174,12 @@ LORA_API int lora_pool_target_offsets(const lora_pool *pool, int target,
 /* ---------------------------------------------------------- the workspace */
 
 /*
- * Device workspace for batches of up to max_tokens rows (the call's T): holds
- * the plan (rows grouped by adapter, work items).  The target argument is
- * accepted for future per-target needs; the size does not depend on it today.
+ * Device workspace for calls on `target` with up to max_tokens rows (the
+ * call's T): the plan (rows grouped by adapter, work items, tensor-core
+ * tiles), then, where the tensor-core segment path can serve the target, the
+ * fp32 partial V of each k-slice of d_in (T x slices x rank bound x 4 bytes).
+ * A workspace shared by several targets takes the largest of their sizes.
+ * Calls with a smaller workspace return LORA_ERR_WORKSPACE.
  */
 LORA_API size_t lora_workspace_bytes(const lora_pool *pool, int target, int max_tokens);
 

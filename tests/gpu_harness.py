@@ -96,7 +96,8 @@ class DevicePool:
 
 
 def workspace(pool: DevicePool, T: int) -> torch.Tensor:
-    n = L.lora_workspace_bytes(pool.pool, 0, T)
+    """A workspace good for every target of the pool (the largest size)."""
+    n = max(L.lora_workspace_bytes(pool.pool, t, T) for t in range(len(pool.w.targets)))
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=pool.device)
 
 

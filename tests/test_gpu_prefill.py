@@ -1,6 +1,7 @@
 """GPU parity of the segment (prefill) path: long segments on the tensor cores
-(tcgen05 MMA, TMA tiles, 128-row tiles split over a cluster), short segments
-on the decode kernel, against the fp64 oracle on the same seeded inputs.
+(tcgen05 MMA, TMA tiles; 128-row tiles, a shrink launch over k-slices and an
+expand launch over column groups), short segments on the decode kernel,
+against the fp64 oracle on the same seeded inputs.
 
 Bound: max |y_gpu - y_ref| <= 4e-3 * max |y_ref|, with the base output and
 with y = 0 (delta alone); rows outside every segment and rows of segments
@@ -78,7 +79,7 @@ def test_prefill_config_uses_tensor_cores_and_matches(cuda_device):
     with DevicePool(w, cuda_device) as pool:
         n0 = L.lora_kernel_launches()
         got = _run_segments(pool, w, 0, w.x(0), w.y_in(0), w.seg_offsets, w.seg_slot)
-        assert L.lora_kernel_launches() - n0 == 3          # plan, decode (short segments), tensor-core
+        assert L.lora_kernel_launches() - n0 == 4  # plan, decode (short segments), tensor-core shrink, expand
         ref, _ = oracle_y(w, 0, w.x(0), w.y_in(0), w.ids)
         assert_close(got, ref, what="config 3")
         got0 = _run_segments(pool, w, 0, w.x(0), np.zeros_like(w.y_in(0)), w.seg_offsets, w.seg_slot)
