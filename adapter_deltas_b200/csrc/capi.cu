@@ -131,6 +131,11 @@ int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ld
   if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
   if (!scales || !ids) return LORA_ERR_INVALID_ARG;
   if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  if (T <= kFusedMaxT) {  // one launch: the delta kernel groups the rows itself
+    DeviceGuard g(p->device);
+    return launch_decode_ids(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, ids, T,
+                             static_cast<cudaStream_t>(stream));
+  }
   if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
   return lora_apply_plan(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, stream);
 }
@@ -155,6 +160,11 @@ int lora_shrink(lora_pool *p, int target, const void *x, int ldx, const int32_t 
   if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
   if (!ids || !v || ldv < p->r_max) return LORA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(v) & 3u) return LORA_ERR_ALIGNMENT;
+  if (T <= kFusedMaxT) {
+    DeviceGuard g(p->device);
+    return launch_decode_ids(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, ldv, ids, T,
+                             static_cast<cudaStream_t>(stream));
+  }
   if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
   DeviceGuard g(p->device);
   return launch_decode(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, ldv, T, ws,
@@ -168,6 +178,11 @@ int lora_expand(lora_pool *p, int target, const float *v, int ldv, void *y, int 
   if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
   if (!ids || !v || !scales || ldv < p->r_max) return LORA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(v) & 3u) return LORA_ERR_ALIGNMENT;
+  if (T <= kFusedMaxT) {
+    DeviceGuard g(p->device);
+    return launch_decode_ids(p, kExpandOnly, target, nullptr, 0, y, ldy, scales, const_cast<float *>(v), ldv, ids,
+                             T, static_cast<cudaStream_t>(stream));
+  }
   if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
   DeviceGuard g(p->device);
   return launch_decode(p, kExpandOnly, target, nullptr, 0, y, ldy, scales, const_cast<float *>(v), ldv, T, ws,

@@ -35,6 +35,7 @@ constexpr int kDecodeThreads = kConsumerThreads;
 constexpr int kClusterCtas = 8;      // CTAs that split one work item (portable cluster)
 constexpr int kMaxStages = 4;        // pipeline depth of the decode kernel
 constexpr int kItemSlots = 8;        // items a warp's copies may run ahead of its compute
+constexpr int kFusedMaxT = 256;      // batches up to this size are grouped inside the decode kernel
 
 extern std::atomic<uint64_t> g_launches;
 
@@ -294,6 +295,10 @@ int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx,
 int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
                         const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
                         int items_hdr);
+// Decode launch that groups ids[0 .. T) itself (T <= kFusedMaxT): no plan
+// kernel and no workspace.
+int launch_decode_ids(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
+                      const float *scales, float *v, int ldv, const int32_t *ids, int T, cudaStream_t st);
 struct PrefillGeometry {
   int r_cap, kb_per, n_ks, n_stages, n_groups, smem_sh, smem_ex;
 };

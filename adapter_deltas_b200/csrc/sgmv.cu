@@ -25,6 +25,7 @@
 // independent of the other rows of the batch).  The expand then adds
 // scale * (B v) to its y slice in fp32 and stores bf16 (round to nearest even).
 #include <algorithm>
+#include <climits>
 
 #include "internal.cuh"
 
@@ -50,6 +51,8 @@ struct DecodeArgs {
   int tile_vecs;  // 16-byte vectors per staged row (64 or 32)
   int row_pitch;  // bytes between staged rows (tile_vecs * 16 + 16)
   int items_hdr;  // header word holding the item count to process
+  const int32_t *ids;  // non-null: group the rows of ids[0 .. T) inside the kernel (T <= kFusedMaxT)
+  int T;
 };
 
 // Copy `bytes` of slot's logical range starting at `off` into dst, cut at
@@ -297,7 +300,12 @@ struct DecodeSmem {
   ItemInfo *info;  // [kConsumerWarps][kItemSlots]
   float *red;      // [kConsumerWarps][kItemRows * r_max]: the warps' shrink partials
   float *v, *recv;
+  // in-kernel grouping of an index vector (kFusedMaxT rows)
+  int *f_key, *f_perm, *f_warp;
+  int4 *f_info, *f_items;
 };
+
+constexpr int kFusedBytes = kFusedMaxT * (4 + 4 + 16 + 16) + 64;
 
 __device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeArgs &a) {
   DecodeSmem S;
@@ -310,8 +318,81 @@ __device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeAr
   S.info = reinterpret_cast<ItemInfo *>(p); p += kConsumerWarps * kItemSlots * sizeof(ItemInfo);
   S.red = reinterpret_cast<float *>(p); p += kConsumerWarps * kItemRows * a.r_max * 4;
   S.v = reinterpret_cast<float *>(p); p += kItemRows * kRMax * 4;
-  S.recv = reinterpret_cast<float *>(p);  // [2][C][kItemRows * r_max]
+  S.recv = reinterpret_cast<float *>(p); p += 2 * kClusterCtas * kItemRows * a.r_max * 4;  // [2][C][kItemRows * r_max]
+  S.f_info = reinterpret_cast<int4 *>(p); p += kFusedMaxT * 16;
+  S.f_items = reinterpret_cast<int4 *>(p); p += kFusedMaxT * 16;
+  S.f_key = reinterpret_cast<int *>(p); p += kFusedMaxT * 4;
+  S.f_perm = reinterpret_cast<int *>(p); p += kFusedMaxT * 4;
+  S.f_warp = reinterpret_cast<int *>(p);
   return S;
+}
+
+// Grouping of an index vector inside the kernel, for batches of at most
+// kFusedMaxT rows (every CTA computes the same result): the rows of each
+// adapter in ascending row order, adapters in ascending slot order, cut into
+// items of at most kItemRows rows -- the same items, in the same order, as
+// the plan kernel writes.  Row t's place is found by counting the rows with
+// a smaller slot, or the same slot and a smaller row.  Returns the item
+// count; S.f_perm / S.f_items hold the row order and the items.
+static_assert(kFusedMaxT == kDecodeThreads, "one row of the index vector per thread");
+__device__ int fused_plan(const DecodeArgs &a, const DecodeSmem &S, int tid) {
+  const int T = a.T;
+  int key = INT_MAX, bad = 0;
+  if (tid < T) {
+    const int id = a.ids[tid];
+    if (id != -1) {
+      if (id < -1 || id >= a.pool.n_slots) bad = 1;
+      else if (!a.pool.loaded[id]) bad = 2;
+      else key = id;
+    }
+  }
+  S.f_key[tid] = key;
+  const int any_bad = __syncthreads_or(bad == 1);
+  const int any_empty = __syncthreads_or(bad == 2);
+  if (blockIdx.x == 0 && tid == 0) {
+    if (any_bad) set_status(a.status, LORA_ERR_BAD_ID);
+    else if (any_empty) set_status(a.status, LORA_ERR_NOT_LOADED);
+  }
+  const bool valid = key != INT_MAX;
+  int less = 0, same = 0, same_before = 0;
+  if (valid) {
+    for (int u = 0; u < T; ++u) {
+      const int k = S.f_key[u];
+      less += k < key;
+      same += k == key;
+      same_before += (k == key) & (u < tid);
+    }
+  }
+  const int n_valid = __syncthreads_count(valid);
+  if (valid) {
+    const int pos = less + same_before;
+    S.f_perm[pos] = tid;
+    S.f_info[pos] = make_int4(key, same_before, same, 0);
+  }
+  __syncthreads();
+  // item starts: sorted positions whose offset inside their segment is a
+  // multiple of kItemRows; a block scan numbers them in position order
+  const int4 inf = tid < n_valid ? S.f_info[tid] : make_int4(0, 1, 0, 0);
+  const int flag = (tid < n_valid && inf.y % kItemRows == 0) ? 1 : 0;
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = flag;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) S.f_warp[warp] = incl;
+  __syncthreads();
+  int base = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kDecodeThreads / 32; ++w) {
+    const int c = S.f_warp[w];
+    base += w < warp ? c : 0;
+    total += c;
+  }
+  if (flag) S.f_items[base + incl - 1] = make_int4(inf.x, tid, min(kItemRows, inf.z - inf.y), 0);
+  __syncthreads();
+  return total;
 }
 
 // Where a warp's next copies come from: the item it is copying, with the
@@ -357,10 +438,22 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   griddep_wait();
   griddep_launch_dependents();
 
-  // the header and this cluster's first item are read together (the items
-  // array always has room for cid, whatever the count)
-  const int n_items = a.hdr[a.items_hdr];
-  const int4 d0 = a.items[cid];
+  // The item list: grouped here from the index vector, or the plan's (its
+  // header and this cluster's first item are read together: the items array
+  // always has room for cid, whatever the count).
+  const int4 *items = a.items;
+  const int32_t *perm = a.perm;
+  int n_items;
+  int4 d0;
+  if (a.ids) {
+    n_items = fused_plan(a, S, tid);
+    items = S.f_items;
+    perm = S.f_perm;
+    d0 = cid < n_items ? items[cid] : make_int4(0, 0, 0, 0);
+  } else {
+    n_items = a.hdr[a.items_hdr];
+    d0 = a.items[cid];
+  }
   const int nvi = a.d_in / 8, nvo = a.d_out / 8;
   const int per_i = (nvi + C - 1) / C, per_o = (nvo + C - 1) / C;
   const int kv0 = min(crank * per_i, nvi), kv1 = min(kv0 + per_i, nvi);
@@ -381,12 +474,12 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   is.d_next = d0;
   auto resolve = [&](int li) {
     const int4 d = is.d_next;
-    if (li + 1 < my_items) is.d_next = a.items[cid + (li + 1) * ncl];  // lands while this item streams
+    if (li + 1 < my_items) is.d_next = items[cid + (li + 1) * ncl];  // lands while this item streams
     is.slot = d.x;
     is.m = d.z;
     is.r = a.pool.rank[is.slot * a.pool.n_targets + a.target];
     const float scale = a.scales ? a.scales[is.slot] : 0.f;
-    const int my_row = lane < is.m ? a.perm[d.y + lane] : 0;
+    const int my_row = lane < is.m ? perm[d.y + lane] : 0;
     const uint8_t *wa[2] = {nullptr, nullptr}, *wb[2] = {nullptr, nullptr};
     bool sa = false, sb = false;
 #pragma unroll
@@ -611,7 +704,8 @@ static int decode_smem_bytes(int r_max, int *stage_bytes, int *n_stages) {
   decode_geometry(r_max, &tv, &pitch, n_stages);
   *stage_bytes = (r_max + kItemRows) * pitch;
   return *n_stages * *stage_bytes + (2 * kMaxStages + 2) * 8 + 32 + kConsumerWarps * kItemSlots * (int)sizeof(ItemInfo) +
-         kConsumerWarps * kItemRows * r_max * 4 + kItemRows * kRMax * 4 + 2 * kClusterCtas * kItemRows * r_max * 4;
+         kConsumerWarps * kItemRows * r_max * 4 + kItemRows * kRMax * 4 + 2 * kClusterCtas * kItemRows * r_max * 4 +
+         kFusedBytes;
 }
 
 // Rank rows per warp of the shrink: the smallest power of two with
@@ -704,11 +798,9 @@ int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx,
   return launch_decode_items(pool, mode, target, x, ldx, y, ldy, scales, v, ldv, T, ws, st, kHdrItems);
 }
 
-int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
-                        const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
-                        int items_hdr) {
-  PlanLayout L = plan_layout(T);
-  PlanView pv = plan_view(const_cast<void *>(ws), L);
+static int launch_decode_args(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
+                              const float *scales, float *v, int ldv, int T, const void *ws, const int32_t *ids,
+                              cudaStream_t st, int items_hdr) {
   DecodeArgs a;
   a.pool = pool->view();
   a.target = target;
@@ -722,9 +814,19 @@ int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, in
   a.y = static_cast<uint16_t *>(y);
   a.ldy = ldy;
   a.scales = scales;
-  a.hdr = pv.hdr;
-  a.perm = pv.perm;
-  a.items = pv.items;
+  if (ids) {
+    a.hdr = nullptr;
+    a.perm = nullptr;
+    a.items = nullptr;
+  } else {
+    PlanLayout L = plan_layout(T);
+    PlanView pv = plan_view(const_cast<void *>(ws), L);
+    a.hdr = pv.hdr;
+    a.perm = pv.perm;
+    a.items = pv.items;
+  }
+  a.ids = ids;
+  a.T = T;
   a.v = v;
   a.ldv = ldv;
   a.status = pool->d_status;
@@ -750,6 +852,18 @@ int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, in
     return LORA_ERR_CUDA;
   }
   return LORA_OK;
+}
+
+int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
+                        const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
+                        int items_hdr) {
+  return launch_decode_args(pool, mode, target, x, ldx, y, ldy, scales, v, ldv, T, ws, nullptr, st, items_hdr);
+}
+
+int launch_decode_ids(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
+                      const float *scales, float *v, int ldv, const int32_t *ids, int T, cudaStream_t st) {
+  if (T < 1 || T > kFusedMaxT) return LORA_ERR_INVALID_ARG;
+  return launch_decode_args(pool, mode, target, x, ldx, y, ldy, scales, v, ldv, T, nullptr, ids, st, kHdrItems);
 }
 
 }  // namespace lora

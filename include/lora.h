@@ -252,7 +252,13 @@ LORA_API int lora_apply_plan(lora_pool *pool, int target, const void *x, int ldx
 
 /* ------------------------------------------------------- one-call entry */
 
-/* lora_plan_ids followed by lora_apply_plan. */
+/*
+ * lora_plan_ids followed by lora_apply_plan, with the same result.  Batches
+ * of at most 256 rows take one launch instead: the delta kernel groups the
+ * rows itself (the same segments and items as lora_plan_ids), and ws is then
+ * not written -- callers that reuse a plan across targets call lora_plan_ids
+ * and lora_apply_plan.  ws / ws_bytes are checked the same way either way.
+ */
 LORA_API int lora_apply(lora_pool *pool, int target, const void *x, int ldx, void *y,
                int ldy, const int32_t *ids, const float *scales, int T,
                void *ws, size_t ws_bytes, void *stream);
@@ -270,7 +276,8 @@ LORA_API int lora_apply_segments(lora_pool *pool, int target, const void *x, int
  *   and leaves other rows of v untouched.
  *   lora_expand adds scales[a] * B_a v[t, 0:r_a] to y[t] in place.
  * lora_shrink followed by lora_expand gives bit-identical y to lora_apply:
- * both use the same reduction order.
+ * both use the same reduction order.  Like lora_apply, batches of at most
+ * 256 rows are grouped inside the kernel and leave ws unwritten.
  */
 LORA_API int lora_shrink(lora_pool *pool, int target, const void *x, int ldx,
                 const int32_t *ids, int T, float *v, int ldv, void *ws,
