@@ -179,42 +179,53 @@ __device__ __forceinline__ void expand_prepare(const float *s_v, int r, int m, E
 }
 
 template <int JB>
+__device__ __forceinline__ void expand_group(uint32_t buf_u, const uint8_t *yb, uint32_t zero_u, int pitch, int wv,
+                                             int v_lo, int r, int m, const ExpandA<JB> &A, float scale,
+                                             const int *s_rows, const DecodeArgs &a, int lane, int cg) {
+  const int g = lane >> 2, t = lane & 3;
+  const int bj = (lane & 7) + ((lane >> 3) & 1) * 8, bn = (lane >> 4) * 16;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
+    // ranks j >= r read 16 zero bytes: their V is zero and stale weights
+    // (possibly not finite) must not meet it
+    const int j = 16 * ks + bj;
+    uint32_t b[4];
+    ldsm_x4_t(j < r ? buf_u + j * pitch + cg * 32 + bn : zero_u + bn, b);
+    mma_bf16_16816(acc[0], A.hi[ks], b[0], b[1]);
+    mma_bf16_16816(acc[1], A.hi[ks], b[2], b[3]);
+    mma_bf16_16816(acc[0], A.lo[ks], b[0], b[1]);
+    mma_bf16_16816(acc[1], A.lo[ks], b[2], b[3]);
+  }
+  const int n_nt = 2 * cg + 1 < wv ? 2 : 1;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    if (nt >= n_nt) break;
+    const int col = cg * 16 + nt * 8 + 2 * t;  // within the tile
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int i = g + hr * 8;
+      if (i < m) {
+        const uint32_t yv = *reinterpret_cast<const uint32_t *>(yb + i * pitch + col * 2);
+        const uint32_t o = pack_bf16x2(fmaf(scale, acc[nt][2 * hr], bf16_lo(yv)),
+                                       fmaf(scale, acc[nt][2 * hr + 1], bf16_hi(yv)));
+        *reinterpret_cast<uint32_t *>(a.y + (long long)s_rows[i] * a.ldy + (long long)v_lo * 8 + col) = o;
+      }
+    }
+  }
+}
+
+// The warp takes the 16-column groups warp, warp + 8, ... two at a time
+// (independent MMA chains side by side).
+template <int JB>
 __device__ __forceinline__ void expand_mma(uint32_t buf_u, const uint8_t *yb, uint32_t zero_u, int pitch, int wv,
                                            int v_lo, int r, int m, const ExpandA<JB> &A, float scale,
                                            const int *s_rows, const DecodeArgs &a, int lane, int warp) {
-  const int g = lane >> 2, t = lane & 3;
   const int groups = (wv + 1) / 2;  // 16-column groups (an odd last vector is half a group)
-  const int bj = (lane & 7) + ((lane >> 3) & 1) * 8, bn = (lane >> 4) * 16;
-  for (int cg = warp; cg < groups; cg += kConsumerWarps) {
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
-      // ranks j >= r read 16 zero bytes: their V is zero and stale weights
-      // (possibly not finite) must not meet it
-      const int j = 16 * ks + bj;
-      uint32_t b[4];
-      ldsm_x4_t(j < r ? buf_u + j * pitch + cg * 32 + bn : zero_u + bn, b);
-      mma_bf16_16816(acc[0], A.hi[ks], b[0], b[1]);
-      mma_bf16_16816(acc[0], A.lo[ks], b[0], b[1]);
-      mma_bf16_16816(acc[1], A.hi[ks], b[2], b[3]);
-      mma_bf16_16816(acc[1], A.lo[ks], b[2], b[3]);
-    }
-    const int n_nt = 2 * cg + 1 < wv ? 2 : 1;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      if (nt >= n_nt) break;
-      const int col = cg * 16 + nt * 8 + 2 * t;  // within the tile
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int i = g + hr * 8;
-        if (i < m) {
-          const uint32_t yv = *reinterpret_cast<const uint32_t *>(yb + i * pitch + col * 2);
-          const uint32_t o = pack_bf16x2(fmaf(scale, acc[nt][2 * hr], bf16_lo(yv)),
-                                         fmaf(scale, acc[nt][2 * hr + 1], bf16_hi(yv)));
-          *reinterpret_cast<uint32_t *>(a.y + (long long)s_rows[i] * a.ldy + (long long)v_lo * 8 + col) = o;
-        }
-      }
-    }
+  for (int cg = warp; cg < groups; cg += 2 * kConsumerWarps) {
+    expand_group<JB>(buf_u, yb, zero_u, pitch, wv, v_lo, r, m, A, scale, s_rows, a, lane, cg);
+    if (cg + kConsumerWarps < groups)
+      expand_group<JB>(buf_u, yb, zero_u, pitch, wv, v_lo, r, m, A, scale, s_rows, a, lane, cg + kConsumerWarps);
   }
 }
 
@@ -301,11 +312,11 @@ struct DecodeSmem {
   float *red;      // [kConsumerWarps][kItemRows * r_max]: the warps' shrink partials
   float *v, *recv;
   // in-kernel grouping of an index vector (kFusedMaxT rows)
-  int *f_key, *f_perm, *f_warp;
-  int4 *f_info, *f_items;
+  int *f_key, *f_perm, *f_warp, *f_items;
+  int4 *f_info, *f_slot;
 };
 
-constexpr int kFusedBytes = kFusedMaxT * (4 + 4 + 16 + 16) + 64;
+constexpr int kFusedBytes = kFusedMaxT * (4 + 4 + 4 + 16 + 16) + 64;
 
 __device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeArgs &a) {
   DecodeSmem S;
@@ -320,7 +331,8 @@ __device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeAr
   S.v = reinterpret_cast<float *>(p); p += kItemRows * kRMax * 4;
   S.recv = reinterpret_cast<float *>(p); p += 2 * kClusterCtas * kItemRows * a.r_max * 4;  // [2][C][kItemRows * r_max]
   S.f_info = reinterpret_cast<int4 *>(p); p += kFusedMaxT * 16;
-  S.f_items = reinterpret_cast<int4 *>(p); p += kFusedMaxT * 16;
+  S.f_slot = reinterpret_cast<int4 *>(p); p += kFusedMaxT * 16;
+  S.f_items = reinterpret_cast<int *>(p); p += kFusedMaxT * 4;
   S.f_key = reinterpret_cast<int *>(p); p += kFusedMaxT * 4;
   S.f_perm = reinterpret_cast<int *>(p); p += kFusedMaxT * 4;
   S.f_warp = reinterpret_cast<int *>(p);
@@ -329,38 +341,61 @@ __device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeAr
 
 // Grouping of an index vector inside the kernel, for batches of at most
 // kFusedMaxT rows (every CTA computes the same result): the rows of each
-// adapter in ascending row order, adapters in ascending slot order, cut into
-// items of at most kItemRows rows -- the same items, in the same order, as
-// the plan kernel writes.  Row t's place is found by counting the rows with
-// a smaller slot, or the same slot and a smaller row.  Returns the item
-// count; S.f_perm / S.f_items hold the row order and the items.
-static_assert(kFusedMaxT == kDecodeThreads, "one row of the index vector per thread");
-__device__ int fused_plan(const DecodeArgs &a, const DecodeSmem &S, int tid) {
+// slot in ascending row order, slots in ascending order, cut into items of
+// at most kItemRows rows -- the plan kernel's items, in the same order, plus
+// items for slots that hold no adapter (rank 0: they change no row; the
+// resolve step reports them).  Row t's place is found by counting the rows
+// with a smaller slot, or the same slot and a smaller index.  Each row's
+// thread also loads what resolving its slot needs -- rank, scale and the
+// physical pages of this CTA's A and B^T slices (-1 when the slices do not
+// lie on one page) -- while the rows are being ranked; the first row of each
+// item keeps them in S.f_slot.  Items are packed as slot | start << 14 |
+// m << 22.  Returns the item count; *any_bad is set when some id lies
+// outside [-1, n_slots).
+struct SliceGeo {
+  long long a_first, a_last, b_first, b_last;  // logical byte range of the slices (first < 0: none)
+};
+
+__device__ __forceinline__ int slice_page(const PoolView &p, int slot, long long first, long long last) {
+  if (first < 0) return -1;
+  const long long pf = p.log2_page < 0 ? 0 : first >> p.log2_page;
+  const long long pl = p.log2_page < 0 ? 0 : last >> p.log2_page;
+  return pf == pl ? __ldg(p.pt + (long long)slot * p.pps + pf) : -1;
+}
+
+__device__ int fused_plan(const DecodeArgs &a, const DecodeSmem &S, int tid, const SliceGeo &geo, int *any_bad) {
   const int T = a.T;
   int key = INT_MAX, bad = 0;
+  int4 sinfo = make_int4(0, -1, -1, 0);
   if (tid < T) {
     const int id = a.ids[tid];
     if (id != -1) {
-      if (id < -1 || id >= a.pool.n_slots) bad = 1;
-      else if (!a.pool.loaded[id]) bad = 2;
-      else key = id;
+      if (id < -1 || id >= a.pool.n_slots) {
+        bad = 1;
+      } else {
+        key = id;
+        const PoolView &p = a.pool;
+        sinfo.x = p.rank[(long long)id * p.n_targets + a.target];
+        sinfo.y = slice_page(p, id, geo.a_first, geo.a_last);
+        sinfo.z = slice_page(p, id, geo.b_first, geo.b_last);
+        sinfo.w = a.scales ? __float_as_int(a.scales[id]) : 0;
+      }
     }
   }
   S.f_key[tid] = key;
-  const int any_bad = __syncthreads_or(bad == 1);
-  const int any_empty = __syncthreads_or(bad == 2);
-  if (blockIdx.x == 0 && tid == 0) {
-    if (any_bad) set_status(a.status, LORA_ERR_BAD_ID);
-    else if (any_empty) set_status(a.status, LORA_ERR_NOT_LOADED);
-  }
+  *any_bad = __syncthreads_or(bad);
+  if (blockIdx.x == 0 && tid == 0 && *any_bad) set_status(a.status, LORA_ERR_BAD_ID);
   const bool valid = key != INT_MAX;
   int less = 0, same = 0, same_before = 0;
   if (valid) {
-    for (int u = 0; u < T; ++u) {
-      const int k = S.f_key[u];
-      less += k < key;
-      same += k == key;
-      same_before += (k == key) & (u < tid);
+    const int4 *k4 = reinterpret_cast<const int4 *>(S.f_key);  // keys past T are INT_MAX
+    for (int u4 = 0; u4 < (T + 3) / 4; ++u4) {
+      const int4 k = k4[u4];
+      const int u = 4 * u4;
+      less += (k.x < key) + (k.y < key) + (k.z < key) + (k.w < key);
+      same += (k.x == key) + (k.y == key) + (k.z == key) + (k.w == key);
+      same_before += ((k.x == key) & (u < tid)) + ((k.y == key) & (u + 1 < tid)) + ((k.z == key) & (u + 2 < tid)) +
+                     ((k.w == key) & (u + 3 < tid));
     }
   }
   const int n_valid = __syncthreads_count(valid);
@@ -368,6 +403,7 @@ __device__ int fused_plan(const DecodeArgs &a, const DecodeSmem &S, int tid) {
     const int pos = less + same_before;
     S.f_perm[pos] = tid;
     S.f_info[pos] = make_int4(key, same_before, same, 0);
+    if (same_before % kItemRows == 0) S.f_slot[pos] = sinfo;
   }
   __syncthreads();
   // item starts: sorted positions whose offset inside their segment is a
@@ -390,9 +426,13 @@ __device__ int fused_plan(const DecodeArgs &a, const DecodeSmem &S, int tid) {
     base += w < warp ? c : 0;
     total += c;
   }
-  if (flag) S.f_items[base + incl - 1] = make_int4(inf.x, tid, min(kItemRows, inf.z - inf.y), 0);
+  if (flag) S.f_items[base + incl - 1] = inf.x | (tid << 14) | (min(kItemRows, inf.z - inf.y) << 22);
   __syncthreads();
   return total;
+}
+
+__device__ __forceinline__ int4 unpack_item(int v) {
+  return make_int4(v & 0x3FFF, (v >> 14) & 0xFF, (v >> 22) & 0x1F, 0);
 }
 
 // Where a warp's next copies come from: the item it is copying, with the
@@ -423,7 +463,7 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&S.full[s], kConsumerThreads);  // every lane arrives once its copies of the tile landed
+      mbar_init(&S.full[s], kConsumerWarps);    // every warp announces its rows' bytes; the copies count them down
       mbar_init(&S.empty[s], kConsumerWarps);   // every warp arrives once it is done with the tile
     }
     mbar_init(&S.recv_full[0], 1);
@@ -441,23 +481,34 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   // The item list: grouped here from the index vector, or the plan's (its
   // header and this cluster's first item are read together: the items array
   // always has room for cid, whatever the count).
-  const int4 *items = a.items;
-  const int32_t *perm = a.perm;
-  int n_items;
-  int4 d0;
-  if (a.ids) {
-    n_items = fused_plan(a, S, tid);
-    items = S.f_items;
-    perm = S.f_perm;
-    d0 = cid < n_items ? items[cid] : make_int4(0, 0, 0, 0);
-  } else {
-    n_items = a.hdr[a.items_hdr];
-    d0 = a.items[cid];
-  }
   const int nvi = a.d_in / 8, nvo = a.d_out / 8;
   const int per_i = (nvi + C - 1) / C, per_o = (nvo + C - 1) / C;
   const int kv0 = min(crank * per_i, nvi), kv1 = min(kv0 + per_i, nvi);
   const int nv0 = min(crank * per_o, nvo), nv1 = min(nv0 + per_o, nvo);
+  const bool fused = a.ids != nullptr;
+  const int32_t *perm = a.perm;
+  int n_items;
+  int4 d0;
+  int any_bad = 1;  // (plan path: the plan kernel reported empty slots itself)
+  if (fused) {
+    SliceGeo geo;
+    geo.a_first = geo.b_first = -1;
+    geo.a_last = geo.b_last = -1;
+    if (MODE != kExpandOnly && kv1 > kv0) {
+      geo.a_first = a.a_off + (long long)kv0 * 16;
+      geo.a_last = a.a_off + ((long long)(a.r_max - 1) * a.d_in + (long long)kv1 * 8) * 2 - 1;
+    }
+    if (MODE != kShrinkOnly && nv1 > nv0) {
+      geo.b_first = a.bt_off + (long long)nv0 * 16;
+      geo.b_last = a.bt_off + ((long long)(a.r_max - 1) * a.d_out + (long long)nv1 * 8) * 2 - 1;
+    }
+    n_items = fused_plan(a, S, tid, geo, &any_bad);
+    perm = S.f_perm;
+    d0 = cid < n_items ? unpack_item(S.f_items[cid]) : make_int4(0, 0, 0, 0);
+  } else {
+    n_items = a.hdr[a.items_hdr];
+    d0 = a.items[cid];
+  }
   const int nk = (MODE == kExpandOnly) ? 0 : (per_i + TV - 1) / TV;
   const int nn = (MODE == kShrinkOnly) ? 0 : (per_o + TV - 1) / TV;
   const int tpi = nk + nn;
@@ -474,11 +525,21 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   is.d_next = d0;
   auto resolve = [&](int li) {
     const int4 d = is.d_next;
-    if (li + 1 < my_items) is.d_next = items[cid + (li + 1) * ncl];  // lands while this item streams
+    if (li + 1 < my_items)  // lands while this item streams
+      is.d_next = fused ? unpack_item(S.f_items[cid + (li + 1) * ncl]) : a.items[cid + (li + 1) * ncl];
     is.slot = d.x;
     is.m = d.z;
-    is.r = a.pool.rank[is.slot * a.pool.n_targets + a.target];
-    const float scale = a.scales ? a.scales[is.slot] : 0.f;
+    // rank, scale and the slices' physical pages: gathered during the
+    // in-kernel grouping, else read now (one level of loads, all together)
+    int4 sinfo;
+    if (fused) {
+      sinfo = S.f_slot[d.y];
+    } else {
+      sinfo.x = a.pool.rank[is.slot * a.pool.n_targets + a.target];
+      sinfo.y = sinfo.z = -1;
+      sinfo.w = a.scales ? __float_as_int(a.scales[is.slot]) : 0;
+    }
+    const float scale = __int_as_float(sinfo.w);
     const int my_row = lane < is.m ? perm[d.y + lane] : 0;
     const uint8_t *wa[2] = {nullptr, nullptr}, *wb[2] = {nullptr, nullptr};
     bool sa = false, sb = false;
@@ -488,17 +549,32 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
       if (j < a.r_max) {
         long long room;
         if (MODE != kExpandOnly && wlen_a > 0) {
-          wa[h] = pool_addr(a.pool, is.slot, a.a_off + ((long long)j * a.d_in + (long long)kv0 * 8) * 2, &room);
-          sa |= (j < is.r) && (wa[h] == nullptr || room < wlen_a);
+          const long long off = a.a_off + ((long long)j * a.d_in + (long long)kv0 * 8) * 2;
+          if (sinfo.y >= 0) {
+            wa[h] = a.pool.base + (long long)sinfo.y * a.pool.page_bytes +
+                    (a.pool.log2_page < 0 ? off : off & (a.pool.page_bytes - 1));
+          } else {
+            wa[h] = pool_addr(a.pool, is.slot, off, &room);
+            sa |= (j < sinfo.x) && (wa[h] == nullptr || room < wlen_a);
+          }
         }
         if (MODE != kShrinkOnly && wlen_b > 0) {
-          wb[h] = pool_addr(a.pool, is.slot, a.bt_off + ((long long)j * a.d_out + (long long)nv0 * 8) * 2, &room);
-          sb |= (j < is.r) && (wb[h] == nullptr || room < wlen_b);
+          const long long off = a.bt_off + ((long long)j * a.d_out + (long long)nv0 * 8) * 2;
+          if (sinfo.z >= 0) {
+            wb[h] = a.pool.base + (long long)sinfo.z * a.pool.page_bytes +
+                    (a.pool.log2_page < 0 ? off : off & (a.pool.page_bytes - 1));
+          } else {
+            wb[h] = pool_addr(a.pool, is.slot, off, &room);
+            sb |= (j < sinfo.x) && (wb[h] == nullptr || room < wlen_b);
+          }
         }
       }
     }
+    is.r = sinfo.x;
     is.split_a = __any_sync(0xffffffffu, sa);
     is.split_b = __any_sync(0xffffffffu, sb);
+    if (!any_bad && lane == 0 && warp == 0 && crank == 0 && is.r == 0 && !a.pool.loaded[is.slot])
+      set_status(a.status, LORA_ERR_NOT_LOADED);  // (in-kernel grouping keeps rows of empty slots)
     is.wa0 = (unsigned long long)wa[0];
     is.wa1 = (unsigned long long)wa[1];
     is.wb0 = (unsigned long long)wb[0];
@@ -516,8 +592,10 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   };
 
   // ---- copy this warp's share of the next tile into `stage`: tile row q
-  // (weight rows first, then activation rows) is copied by warp q % 8, one
-  // 16-byte cp.async per lane, so a row is one coalesced warp instruction.
+  // (weight rows first, then activation rows) belongs to warp q % 8, and lane
+  // q / 8 of that warp moves it with one bulk copy (more only where the row
+  // crosses a page).  The warp first announces its rows' bytes on the stage's
+  // barrier, then the copies count them down as they land.
   auto issue_next = [&](int stage) {
     if (is.tt == 0) resolve(is.li);
     const bool shrink = is.tt < nk;
@@ -526,39 +604,35 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
     const int wv = max(0, min(v_lo + TV, shrink ? kv1 : nv1) - v_lo);
     const int rows = (wv > 0 && is.r > 0 && is.m > 0) ? is.r + is.m : 0;
     uint8_t *buf = S.ring + stage * a.stage_bytes;
-    const bool on0 = lane < wv, on1 = lane + 32 < wv;
     const unsigned long long w0 = shrink ? is.wa0 : is.wb0, w1 = shrink ? is.wa1 : is.wb1;
     const bool split = shrink ? is.split_a : is.split_b;
     const unsigned long long act = shrink ? is.xrow : is.yrow;
-    for (int q = warp; q < rows; q += kConsumerWarps) {
+    const int q = warp + kConsumerWarps * lane;  // this lane's row of the tile
+    const int my_rows = rows > warp ? (rows - warp + kConsumerWarps - 1) / kConsumerWarps : 0;
+    const uint32_t bytes = (uint32_t)wv * 16u;
+    // row start addresses (lane-held by the resolve step) for this lane's row
+    const unsigned long long wsrc_lo = __shfl_sync(0xffffffffu, w0, q & 31);
+    const unsigned long long wsrc_hi = __shfl_sync(0xffffffffu, w1, q & 31);
+    const unsigned long long asrc = __shfl_sync(0xffffffffu, act, (q - is.r) & 31);
+    if (lane == 0) mbar_arrive_expect_tx(&S.full[stage], (uint32_t)my_rows * bytes);
+    __syncwarp();
+    if (lane < my_rows) {
       if (q < is.r) {
-        const unsigned long long base = __shfl_sync(0xffffffffu, q < 32 ? w0 : w1, q & 31);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h == 0 ? !on0 : !on1) continue;
-          const int vec = lane + 32 * h;
-          const uint8_t *src = reinterpret_cast<const uint8_t *>(base) + (long long)t_idx * TV * 16 + vec * 16;
-          if (split) {  // the slice crosses a page: translate this chunk on its own
-            long long room;
-            const long long off = (shrink ? a.a_off + (long long)q * a.d_in * 2 : a.bt_off + (long long)q * a.d_out * 2) +
-                                  (long long)(v_lo + vec) * 16;
-            src = pool_addr(a.pool, is.slot, off, &room);
-            if (src == nullptr) {
-              set_status(a.status, LORA_ERR_NOT_LOADED);
-              src = a.pool.base;
-            }
-          }
-          cp_async16(buf + q * pitch + vec * 16, src);
+        const long long off = (long long)t_idx * TV * 16;
+        if (split) {  // the slice crosses a page: copy it piece by piece
+          const long long loff = (shrink ? a.a_off + (long long)q * a.d_in * 2 : a.bt_off + (long long)q * a.d_out * 2) +
+                                 (long long)v_lo * 16;
+          copy_pool_row(a.pool, is.slot, loff, bytes, buf + q * pitch, &S.full[stage], a.status);
+        } else {
+          bulk_g2s(buf + q * pitch, reinterpret_cast<const uint8_t *>(q < 32 ? wsrc_lo : wsrc_hi) + off, bytes,
+                   &S.full[stage]);
         }
       } else {
         const int i = q - is.r;
-        const unsigned long long base = __shfl_sync(0xffffffffu, act, i);
-        const uint16_t *src = reinterpret_cast<const uint16_t *>(base) + (long long)t_idx * TV * 8;
-        if (on0) cp_async16(buf + act_base + i * pitch + lane * 16, src + lane * 8);
-        if (on1) cp_async16(buf + act_base + i * pitch + (lane + 32) * 16, src + (lane + 32) * 8);
+        bulk_g2s(buf + act_base + i * pitch, reinterpret_cast<const uint8_t *>(asrc) + (long long)t_idx * TV * 16,
+                 bytes, &S.full[stage]);
       }
     }
-    cp_async_arrive(&S.full[stage]);
     if (++is.tt == tpi) {
       is.tt = 0;
       ++is.li;
