@@ -213,6 +213,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ void set_status(int *status, int code) { atomicCAS(status, 0, code); }
 
+// Copy `bytes` of slot's logical range starting at `off` into dst, cut at
+// page boundaries.  A missing page (slot unloaded under our feet) is replaced
+// by page-free reads of the pool base and reported.
+__device__ __forceinline__ void copy_pool_row(const PoolView &pool, int slot, long long off, uint32_t bytes,
+                                              uint8_t *dst, uint64_t *bar, int *status) {
+  while (bytes > 0) {
+    long long room;
+    const uint8_t *src = pool_addr(pool, slot, off, &room);
+    uint32_t n = (uint32_t)min((long long)bytes, room);
+    if (src == nullptr) {
+      set_status(status, LORA_ERR_NOT_LOADED);
+      src = pool.base;
+    }
+    bulk_g2s(dst, src, n, bar);
+    dst += n;
+    off += n;
+    bytes -= n;
+  }
+}
+
+
 // Launch attribute for programmatic dependent launch: the kernel may start
 // while the previous kernel on the stream is still running; it reads that
 // kernel's results only after griddep_wait().  Kernels of this library call

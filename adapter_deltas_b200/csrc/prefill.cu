@@ -48,7 +48,6 @@ constexpr int kShThreads = kShEpiThreads + 64;   // + TMA producer warp + MMA wa
 constexpr int kShMaxStages = 8;
 constexpr int kShMaxBlocks = 16;                  // x blocks (64 columns) per k-slice
 constexpr int kShTmemCols = 32;
-constexpr int kShHeadBlocks = 2;                  // x blocks issued before the adapter slice is on its way
 // expand kernel
 constexpr int kExThreads = 128;                   // warp w: tile rows 32w .. 32w + 31
 constexpr int kGroupCols = kChunkCols;            // d_out columns per unit (one MMA chunk, two y boxes)
@@ -151,8 +150,6 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void st_shared_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
 }
-// Barrier of the shrink kernel's epilogue warps only (named barrier 1).
-__device__ __forceinline__ void sh_epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kShEpiThreads) : "memory"); }
 
 // Address of 16-byte chunk `chunk` of a rank row slice: from the row's start
 // when the slice lies on one page, else through the page table.
@@ -170,14 +167,13 @@ __device__ __forceinline__ const uint8_t *slice_chunk(const PoolView &pool, int 
 
 // ============================================================ shrink kernel
 struct ShSmem {
-  uint8_t *ring, *aw;
-  const uint8_t **arow;
-  uint64_t *full, *empty, *w_full, *w_issued, *sh_done;
+  uint8_t *ring, *aw, *stg;  // x stages; A slice in the MMA layout; A slice rows as copied
+  uint64_t *full, *empty, *w_full, *a_land, *sh_done;
   uint32_t *tmem_slot;
 };
 
 __host__ __device__ inline int sh_smem_bytes(int n_stages, int r_cap, int kb_per) {
-  return 1024 /* alignment slack */ + n_stages * kBoxBytes + r_cap * kb_per * kBoxCols * 2 + kPfRankCap * 8 +
+  return 1024 /* alignment slack */ + n_stages * kBoxBytes + 2 * r_cap * kb_per * kBoxCols * 2 +
          (2 * kShMaxStages + 3) * 8 + 16;
 }
 
@@ -194,12 +190,12 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     uint8_t *p = base;
     S.ring = p; p += NS * kBoxBytes;
     S.aw = p; p += a.r_cap * a.kb_per * kBoxCols * 2;
-    S.arow = reinterpret_cast<const uint8_t **>(p); p += kPfRankCap * 8;
+    S.stg = p; p += a.r_cap * a.kb_per * kBoxCols * 2;
     uint64_t *b = reinterpret_cast<uint64_t *>(p);
     S.full = b; b += kShMaxStages;
     S.empty = b; b += kShMaxStages;
     S.w_full = b++;
-    S.w_issued = b++;
+    S.a_land = b++;
     S.sh_done = b++;
     S.tmem_slot = reinterpret_cast<uint32_t *>(b);
   }
@@ -215,7 +211,7 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
       mbar_init(&S.empty[i], 1);
     }
     mbar_init(S.w_full, kShEpiThreads);
-    mbar_init(S.w_issued, kShEpiWarps);
+    mbar_init(S.a_land, 1);
     mbar_init(S.sh_done, 1);
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&a.tmap_x)) : "memory");
@@ -233,28 +229,22 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
   const uint32_t lbo_a = (uint32_t)(a.r_cap / 8) * 128u;  // k-group stride of the A_a slice
   const uint32_t aw_u = smem_u32(S.aw), ring_u = smem_u32(S.ring);
   uint32_t gbase = 0;   // ring uses so far: use g sits in stage g % NS with phase (g / NS) & 1
-  uint32_t ucount = 0;  // units done (w_full / sh_done phases)
+  uint32_t ucount = 0;  // units multiplied so far (w_full / a_land / sh_done phases)
 
   for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
     const int tile = u / a.n_ks, ks = u - tile * a.n_ks;
+    const int kb0 = ks * a.kb_per, nkb = min(a.kb_per, nkb_all - kb0);
+    if (nkb <= 0) continue;
     const int4 d = a.tiles[tile];
     const int slot = d.x, row0 = d.y, m = d.z;
-    const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
-    const int kb0 = ks * a.kb_per, nkb = min(a.kb_per, nkb_all - kb0);
-    if (r <= 0 || r > a.r_cap || nkb <= 0) {
-      if (r > a.r_cap && tid == 0) set_status(a.status, LORA_ERR_INVALID_ARG);
-      continue;
-    }
-    const int R = (r + 15) & ~15;
-    const uint32_t par = ucount & 1u;
 
     if (warp == kShEpiWarps) {
       // ------------------------------------------------ TMA producer
-      // (after a short head start, the x stream waits until the adapter
-      // slice's copies are issued: they gate the first MMA)
+      // (x depends only on the tile record: the stream starts at once; a
+      // unit whose adapter turns out absent still passes its blocks through
+      // the ring, the MMA warp just does not multiply them)
       if (lane == 0) {
         for (int i = 0; i < nkb; ++i) {
-          if (i == min(kShHeadBlocks, nkb - 1)) pf_wait(S.w_issued, par, a.status, alive);
           const uint32_t g = gbase + i, st = g % NS;
           if (g >= (uint32_t)NS && !pf_wait(&S.empty[st], ((g / NS) - 1) & 1, a.status, alive)) break;
           mbar_arrive_expect_tx(&S.full[st], kBoxBytes);
@@ -262,12 +252,21 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
         }
       }
       __syncwarp();
-    } else if (warp == kShEpiWarps + 1) {
+      gbase += nkb;
+      continue;
+    }
+    const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
+    const bool use = r > 0 && r <= a.r_cap;
+    if (r > a.r_cap && tid == 0) set_status(a.status, LORA_ERR_INVALID_ARG);
+    const int R = (r + 15) & ~15;
+    const uint32_t par = ucount & 1u;
+
+    if (warp == kShEpiWarps + 1) {
       // ------------------------------------------------ MMA issuer
       if (lane == 0) {
-        pf_wait(S.w_full, par, a.status, alive);
+        if (use) pf_wait(S.w_full, par, a.status, alive);
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(R, false);
+        const uint32_t idesc = idesc_bf16(use ? R : 16, false);
         for (int i = 0; i < nkb; ++i) {
           const uint32_t g = gbase + i, st = g % NS;
           pf_wait(&S.full[st], (g / NS) & 1, a.status, alive);
@@ -277,41 +276,37 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
           for (int kk = 0; kk < kBoxCols / 16; ++kk) {
             const uint64_t ad = smem_desc(xa + kk * 32, 16, 1024, 2);
             const uint64_t bd = smem_desc(aw_u + (uint32_t)(i * 4 + kk) * 2 * lbo_a, lbo_a, 128, 0);
-            if (alive) mma_bf16(tmem, ad, bd, idesc, (i | kk) != 0);
+            if (alive && use) mma_bf16(tmem, ad, bd, idesc, (i | kk) != 0);
           }
           mma_commit(&S.empty[st]);  // the stage is free once these MMAs have read it
         }
-        mma_commit(S.sh_done);
+        if (use) mma_commit(S.sh_done);
       }
       __syncwarp();
-    } else {
+    } else if (use) {
       // ------------------------------------------------ epilogue warps
-      // (1) the k-slice of A_a (rows < r; zero rows up to R and columns
-      // beyond d_in) into shared memory in the MMA's K-major core-matrix layout
+      // (1) the k-slice of A_a: rows < r by one bulk copy each (pieces where
+      // a row crosses a page) into a row-major staging area, then moved into
+      // the MMA's K-major core-matrix layout, with zero rows up to R and zero
+      // columns beyond d_in
       const int cols = min(nkb * kBoxCols, a.d_in - kb0 * kBoxCols);
+      const uint32_t row_bytes = (uint32_t)cols * 2u, stg_pitch = (uint32_t)a.kb_per * kBoxCols * 2u;
       const long long row_off0 = a.a_off + (long long)kb0 * kBoxCols * 2;
-      if (tid < r) {
-        long long room;
-        const uint8_t *p = pool_addr(a.pool, slot, row_off0 + (long long)tid * a.d_in * 2, &room);
-        S.arow[tid] = (p && room >= (long long)cols * 2) ? p : nullptr;
+      if (warp == 0) {
+        if (lane == 0) mbar_arrive_expect_tx(S.a_land, (uint32_t)r * row_bytes);
+        __syncwarp();
+        if (lane < r)
+          copy_pool_row(a.pool, slot, row_off0 + (long long)lane * a.d_in * 2, row_bytes, S.stg + lane * stg_pitch,
+                        S.a_land, a.status);
       }
-      sh_epi_sync();
-      const int jl = lane & 7, vo = lane >> 3;  // 8 rank rows x 4 consecutive 16-byte chunks per warp access
+      warp_wait(S.a_land, par, a.status, alive);
       const int kv_n = nkb * (kBoxCols / 8);
-      for (int jg = 0; jg < R / 8; ++jg) {
-        const int j = jg * 8 + jl;
-        const uint8_t *ar = j < r ? S.arow[j] : nullptr;
-        for (int kv = warp * 4 + vo; kv < kv_n; kv += kShEpiWarps * 4) {
-          const uint32_t dst = aw_u + kv * lbo_a + jg * 128 + jl * 16;
-          if (j < r && kv * 8 < cols)
-            cp_async16_pf(dst, slice_chunk(a.pool, slot, ar, row_off0 + (long long)j * a.d_in * 2, kv, a.status));
-          else
-            st_shared_zero16(dst);
-        }
+      for (int idx = tid; idx < R * kv_n; idx += kShEpiThreads) {
+        const int j = idx / kv_n, kv = idx - j * kv_n;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (j < r && kv * 8 < cols) v = *reinterpret_cast<const uint4 *>(S.stg + j * stg_pitch + kv * 16);
+        *reinterpret_cast<uint4 *>(S.aw + kv * lbo_a + (j >> 3) * 128 + (j & 7) * 16) = v;
       }
-      __syncwarp();
-      if (lane == 0) pf_arrive(S.w_issued);
-      cp_async_wait_all();
       fence_async_smem();  // generic-proxy writes -> visible to the MMAs (async proxy)
       tc_fence_before();   // the previous unit's TMEM reads are done
       pf_arrive(S.w_full);
@@ -334,7 +329,7 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
       }
     }
     gbase += nkb;
-    ++ucount;
+    if (use) ++ucount;
   }
 
   tc_fence_before();

@@ -51,29 +51,10 @@ struct DecodeArgs {
   int tile_vecs;  // 16-byte vectors per staged row (64 or 32)
   int row_pitch;  // bytes between staged rows (tile_vecs * 16 + 16)
   int items_hdr;  // header word holding the item count to process
+  int items_cap;  // entries the plan's items array has room for
   const int32_t *ids;  // non-null: group the rows of ids[0 .. T) inside the kernel (T <= kFusedMaxT)
   int T;
 };
-
-// Copy `bytes` of slot's logical range starting at `off` into dst, cut at
-// page boundaries.  A missing page (slot unloaded under our feet) is replaced
-// by page-free reads of the pool base and reported.
-__device__ __forceinline__ void copy_pool_row(const PoolView &pool, int slot, long long off, uint32_t bytes,
-                                              uint8_t *dst, uint64_t *bar, int *status) {
-  while (bytes > 0) {
-    long long room;
-    const uint8_t *src = pool_addr(pool, slot, off, &room);
-    uint32_t n = (uint32_t)min((long long)bytes, room);
-    if (src == nullptr) {
-      set_status(status, LORA_ERR_NOT_LOADED);
-      src = pool.base;
-    }
-    bulk_g2s(dst, src, n, bar);
-    dst += n;
-    off += n;
-    bytes -= n;
-  }
-}
 
 // ------------------------------------------------------------ warp MMA
 // The decode contractions are tiny (an item has at most 16 rows and the rank
@@ -314,6 +295,10 @@ struct DecodeSmem {
   // in-kernel grouping of an index vector (kFusedMaxT rows)
   int *f_key, *f_perm, *f_warp, *f_items;
   int4 *f_info, *f_slot;
+  // this cluster's items, resolved once (reuse the two int4 arrays above
+  // once the grouping is done): (slot, first row, rows, rank) and
+  // (A page, B^T page, scale bits, -)
+  int4 *it_rec, *it_res;
 };
 
 constexpr int kFusedBytes = kFusedMaxT * (4 + 4 + 4 + 16 + 16) + 64;
@@ -336,6 +321,8 @@ __device__ __forceinline__ DecodeSmem decode_carve(uint8_t *smem, const DecodeAr
   S.f_key = reinterpret_cast<int *>(p); p += kFusedMaxT * 4;
   S.f_perm = reinterpret_cast<int *>(p); p += kFusedMaxT * 4;
   S.f_warp = reinterpret_cast<int *>(p);
+  S.it_rec = S.f_info;
+  S.it_res = S.f_slot;
   return S;
 }
 
@@ -443,7 +430,6 @@ struct IssueState {
   int slot, m, r;
   bool split_a, split_b;
   unsigned long long wa0, wa1, wb0, wb1, xrow, yrow;
-  int4 d_next;
 };
 
 template <int MODE, int JB>
@@ -478,37 +464,60 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   griddep_wait();
   griddep_launch_dependents();
 
-  // The item list: grouped here from the index vector, or the plan's (its
-  // header and this cluster's first item are read together: the items array
-  // always has room for cid, whatever the count).
   const int nvi = a.d_in / 8, nvo = a.d_out / 8;
   const int per_i = (nvi + C - 1) / C, per_o = (nvo + C - 1) / C;
   const int kv0 = min(crank * per_i, nvi), kv1 = min(kv0 + per_i, nvi);
   const int nv0 = min(crank * per_o, nvo), nv1 = min(nv0 + per_o, nvo);
+  // logical byte ranges of this CTA's A and B^T slices, rows 0 .. r_max-1
+  SliceGeo geo;
+  geo.a_first = geo.b_first = -1;
+  geo.a_last = geo.b_last = -1;
+  if (MODE != kExpandOnly && kv1 > kv0) {
+    geo.a_first = a.a_off + (long long)kv0 * 16;
+    geo.a_last = a.a_off + ((long long)(a.r_max - 1) * a.d_in + (long long)kv1 * 8) * 2 - 1;
+  }
+  if (MODE != kShrinkOnly && nv1 > nv0) {
+    geo.b_first = a.bt_off + (long long)nv0 * 16;
+    geo.b_last = a.bt_off + ((long long)(a.r_max - 1) * a.d_out + (long long)nv1 * 8) * 2 - 1;
+  }
+
+  // ---- the item list, and this cluster's items resolved once: item k of
+  // the cluster (global index cid + k * ncl) gets its slot, rows, rank, scale
+  // and the physical pages of this CTA's slices, gathered by thread k.
+  // Grouped here from the index vector (all in shared memory), or read from
+  // the plan: its header and thread k's item record are read together (the
+  // items array has room for items_cap entries), then rank, scale and pages.
   const bool fused = a.ids != nullptr;
   const int32_t *perm = a.perm;
   int n_items;
-  int4 d0;
   int any_bad = 1;  // (plan path: the plan kernel reported empty slots itself)
+  int4 rec = make_int4(0, 0, 0, 0), res = make_int4(-1, -1, 0, 0);
   if (fused) {
-    SliceGeo geo;
-    geo.a_first = geo.b_first = -1;
-    geo.a_last = geo.b_last = -1;
-    if (MODE != kExpandOnly && kv1 > kv0) {
-      geo.a_first = a.a_off + (long long)kv0 * 16;
-      geo.a_last = a.a_off + ((long long)(a.r_max - 1) * a.d_in + (long long)kv1 * 8) * 2 - 1;
-    }
-    if (MODE != kShrinkOnly && nv1 > nv0) {
-      geo.b_first = a.bt_off + (long long)nv0 * 16;
-      geo.b_last = a.bt_off + ((long long)(a.r_max - 1) * a.d_out + (long long)nv1 * 8) * 2 - 1;
-    }
     n_items = fused_plan(a, S, tid, geo, &any_bad);
     perm = S.f_perm;
-    d0 = cid < n_items ? unpack_item(S.f_items[cid]) : make_int4(0, 0, 0, 0);
+    const int k = cid + tid * ncl;
+    if (k < n_items) {
+      rec = unpack_item(S.f_items[k]);
+      const int4 sl = S.f_slot[rec.y];
+      rec.w = sl.x;
+      res = make_int4(sl.y, sl.z, sl.w, 0);
+    }
   } else {
+    const int k = cid + tid * ncl;
+    int4 d = make_int4(0, 0, 0, 0);
+    if (k < a.items_cap) d = a.items[k];
     n_items = a.hdr[a.items_hdr];
-    d0 = a.items[cid];
+    if (k < n_items) {
+      const PoolView &p = a.pool;
+      rec = make_int4(d.x, d.y, d.z, p.rank[(long long)d.x * p.n_targets + a.target]);
+      res = make_int4(slice_page(p, d.x, geo.a_first, geo.a_last), slice_page(p, d.x, geo.b_first, geo.b_last),
+                      a.scales ? __float_as_int(a.scales[d.x]) : 0, 0);
+    }
   }
+  __syncthreads();  // (the grouping's arrays are read before they are reused)
+  S.it_rec[tid] = rec;
+  S.it_res[tid] = res;
+  __syncthreads();
   const int nk = (MODE == kExpandOnly) ? 0 : (per_i + TV - 1) / TV;
   const int nn = (MODE == kShrinkOnly) ? 0 : (per_o + TV - 1) / TV;
   const int tpi = nk + nn;
@@ -516,29 +525,28 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   const int total = my_items * tpi;
   const int wlen_a = (kv1 - kv0) * 16, wlen_b = (nv1 - nv0) * 16;
 
-  // ---- resolve an item: one level of loads after the item record, all
-  // issued together; lane L keeps the addresses of rows L / L + 32 of this
-  // CTA's weight slices and of activation row L.
+  // ---- resolve an item from its gathered record (items beyond the first
+  // kDecodeThreads of a cluster, only possible on the plan path, read theirs
+  // now); lane L keeps the addresses of rows L / L + 32 of this CTA's weight
+  // slices and of activation row L.
   IssueState is;
   is.li = 0;
   is.tt = 0;
-  is.d_next = d0;
   auto resolve = [&](int li) {
-    const int4 d = is.d_next;
-    if (li + 1 < my_items)  // lands while this item streams
-      is.d_next = fused ? unpack_item(S.f_items[cid + (li + 1) * ncl]) : a.items[cid + (li + 1) * ncl];
+    int4 d, sinfo;
+    if (li < kDecodeThreads) {
+      d = S.it_rec[li];
+      const int4 rs = S.it_res[li];
+      sinfo = make_int4(d.w, rs.x, rs.y, rs.z);
+    } else {
+      d = a.items[cid + li * ncl];
+      sinfo = make_int4(a.pool.rank[(long long)d.x * a.pool.n_targets + a.target],
+                        slice_page(a.pool, d.x, geo.a_first, geo.a_last),
+                        slice_page(a.pool, d.x, geo.b_first, geo.b_last),
+                        a.scales ? __float_as_int(a.scales[d.x]) : 0);
+    }
     is.slot = d.x;
     is.m = d.z;
-    // rank, scale and the slices' physical pages: gathered during the
-    // in-kernel grouping, else read now (one level of loads, all together)
-    int4 sinfo;
-    if (fused) {
-      sinfo = S.f_slot[d.y];
-    } else {
-      sinfo.x = a.pool.rank[is.slot * a.pool.n_targets + a.target];
-      sinfo.y = sinfo.z = -1;
-      sinfo.w = a.scales ? __float_as_int(a.scales[is.slot]) : 0;
-    }
     const float scale = __int_as_float(sinfo.w);
     const int my_row = lane < is.m ? perm[d.y + lane] : 0;
     const uint8_t *wa[2] = {nullptr, nullptr}, *wb[2] = {nullptr, nullptr};
@@ -899,6 +907,7 @@ static int launch_decode_args(lora_pool *pool, int mode, int target, const void 
     a.perm = pv.perm;
     a.items = pv.items;
   }
+  a.items_cap = ids ? 0 : plan_layout(T).i_max;
   a.ids = ids;
   a.T = T;
   a.v = v;
