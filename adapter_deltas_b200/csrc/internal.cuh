@@ -267,7 +267,8 @@ struct lora_pool {
   int32_t *d_pt = nullptr, *d_rank = nullptr, *d_loaded = nullptr;
   int *d_status = nullptr;
   int decode_smem = 0;
-  int decode_max_clusters = 0;
+  int decode_max_clusters = 0;   // co-resident 8-CTA decode clusters
+  int decode_max_clusters4 = 0;  // co-resident 4-CTA decode clusters
   // Kind of the plan last built into each workspace (1 = index vector,
   // 2 = segments, which may hold tensor-core tiles); kept on the host so that
   // an apply call can pick its kernels without reading the device.

@@ -795,15 +795,15 @@ static int decode_smem_bytes(int r_max, int *stage_bytes, int *n_stages) {
 static int jb_for(int r_max) { return r_max <= 8 ? 1 : r_max <= 16 ? 2 : r_max <= 32 ? 4 : 8; }
 
 template <int MODE, int JB>
-static cudaError_t launch_one(const DecodeArgs &a, int n_clusters, int smem, cudaStream_t st) {
+static cudaError_t launch_one(const DecodeArgs &a, int csize, int n_clusters, int smem, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_clusters * kClusterCtas);
+  cfg.gridDim = dim3(n_clusters * csize);
   cfg.blockDim = dim3(kDecodeThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kClusterCtas;
+  attr[0].val.clusterDim.x = csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1] = pdl_attribute();
@@ -813,12 +813,12 @@ static cudaError_t launch_one(const DecodeArgs &a, int n_clusters, int smem, cud
 }
 
 template <int MODE>
-static cudaError_t launch_mode(const DecodeArgs &a, int jb, int n_clusters, int smem, cudaStream_t st) {
+static cudaError_t launch_mode(const DecodeArgs &a, int jb, int csize, int n_clusters, int smem, cudaStream_t st) {
   switch (jb) {
-    case 1: return launch_one<MODE, 1>(a, n_clusters, smem, st);
-    case 2: return launch_one<MODE, 2>(a, n_clusters, smem, st);
-    case 4: return launch_one<MODE, 4>(a, n_clusters, smem, st);
-    default: return launch_one<MODE, 8>(a, n_clusters, smem, st);
+    case 1: return launch_one<MODE, 1>(a, csize, n_clusters, smem, st);
+    case 2: return launch_one<MODE, 2>(a, csize, n_clusters, smem, st);
+    case 4: return launch_one<MODE, 4>(a, csize, n_clusters, smem, st);
+    default: return launch_one<MODE, 8>(a, csize, n_clusters, smem, st);
   }
 }
 
@@ -851,27 +851,31 @@ int decode_setup(lora_pool *pool) {
   if (set_smem_all<kFused>(smem_cap) != cudaSuccess || set_smem_all<kShrinkOnly>(smem_cap) != cudaSuccess ||
       set_smem_all<kExpandOnly>(smem_cap) != cudaSuccess)
     return LORA_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kClusterCtas);
-  cfg.blockDim = dim3(kDecodeThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kClusterCtas;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  cudaError_t e;
-  switch (jb_for(pool->r_max)) {
-    case 1: e = max_clusters<1>(&n, &cfg); break;
-    case 2: e = max_clusters<2>(&n, &cfg); break;
-    case 4: e = max_clusters<4>(&n, &cfg); break;
-    default: e = max_clusters<8>(&n, &cfg); break;
+  // co-resident clusters of 8 and of 4 CTAs at this pool's shared memory
+  for (int csize : {kClusterCtas, kClusterCtas / 2}) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    cudaError_t e;
+    switch (jb_for(pool->r_max)) {
+      case 1: e = max_clusters<1>(&n, &cfg); break;
+      case 2: e = max_clusters<2>(&n, &cfg); break;
+      case 4: e = max_clusters<4>(&n, &cfg); break;
+      default: e = max_clusters<8>(&n, &cfg); break;
+    }
+    if (e != cudaSuccess || n < 1) return LORA_ERR_CUDA;
+    if (csize == kClusterCtas) pool->decode_max_clusters = n;
+    else pool->decode_max_clusters4 = n;
   }
-  if (e != cudaSuccess || n < 1) return LORA_ERR_CUDA;
-  pool->decode_max_clusters = n;
   return LORA_OK;
 }
 
@@ -921,15 +925,23 @@ static int launch_decode_args(lora_pool *pool, int mode, int target, const void 
   decode_geometry(pool->r_max, &a.tile_vecs, &a.row_pitch, &ns);
   // Items are bounded by min(T, n_slots) segments plus T / kItemRows chunk
   // splits; clusters loop over items, so the grid never exceeds what fits.
+  // A batch that may hold more than twice as many items as there are 8-CTA
+  // clusters takes 4-CTA clusters: twice the items in flight, each split
+  // four ways instead of eight.  (Up to rank 32 only: with rank 64 the
+  // 512-byte rows double the tiles of each item and it measured slower.)
   const long long bound = (long long)std::min(T, pool->n_slots) + (T + kItemRows - 1) / kItemRows;
-  int n_clusters = (int)std::min<long long>(bound, (long long)pool->decode_max_clusters);
+  const bool small_clusters =
+      pool->r_max <= 32 && bound > 2LL * pool->decode_max_clusters && pool->decode_max_clusters4 > 0;
+  const int csize = small_clusters ? kClusterCtas / 2 : kClusterCtas;
+  int n_clusters = (int)std::min<long long>(
+      bound, (long long)(small_clusters ? pool->decode_max_clusters4 : pool->decode_max_clusters));
   if (n_clusters < 1) n_clusters = 1;
   cudaError_t e;
   g_launches.fetch_add(1);
   const int jb = jb_for(pool->r_max);
-  if (mode == kFused) e = launch_mode<kFused>(a, jb, n_clusters, smem, st);
-  else if (mode == kShrinkOnly) e = launch_mode<kShrinkOnly>(a, jb, n_clusters, smem, st);
-  else e = launch_mode<kExpandOnly>(a, jb, n_clusters, smem, st);
+  if (mode == kFused) e = launch_mode<kFused>(a, jb, csize, n_clusters, smem, st);
+  else if (mode == kShrinkOnly) e = launch_mode<kShrinkOnly>(a, jb, csize, n_clusters, smem, st);
+  else e = launch_mode<kExpandOnly>(a, jb, csize, n_clusters, smem, st);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return LORA_ERR_CUDA;

@@ -368,7 +368,7 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     tokens = w.T * world
     value = job_value(w.T, world, ms)
     if segmented:
-        kernel_name = "prefill_kernel"
+        kernel_name = "prefill_kernels"
         kernel_desc = "prefill_kernel (tcgen05) + decode_kernel launch for segments under %d rows" % L.lora_mma_min_rows()
     elif one_launch:
         kernel_name, kernel_desc = "decode_kernel", "decode_kernel<fused> grouping the batch in-kernel (the whole step)"
@@ -388,6 +388,8 @@ def run_b200(args, rank: int, world: int, local_rank: int):
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": traffic_from_profile(kernel_name, "prefill.cu" if segmented else "sgmv.cu",
                                                      args.workload),
+                     "traffic_note": "DRAM bytes of one launch (prefill: shrink + expand launches) from the ncu "
+                                     "summary in profiles/, while its source hash matches",
                      "kernel": kernel_desc, "kernel_us": kernel_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg, "frac_of_8TBps_datasheet": achieved / 8000.0},
         "e2e": {"value": job_value(w.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
