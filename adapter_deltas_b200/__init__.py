@@ -82,6 +82,7 @@ _sig("lora_mma_min_rows", _I, [])
 _sig("lora_apply_plan", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_apply", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_segments", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _I, _P, _Z, _P])
+_sig("lora_apply_multi", _I, [_P, _I, _P, _P, _I, _P, _I, _P, _P, _P, _I, _P, _Z, _P])
 _sig("lora_shrink", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_noalloc", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
@@ -242,6 +243,16 @@ def lora_apply_plan(pool: PoolHandle, target: int, x, y, scales, ws, stream=None
 def lora_apply(pool: PoolHandle, target: int, x, y, ids, scales, ws, stream=None) -> None:
     _check(_lib.lora_apply(pool, target, _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(ids), _ptr(scales),
                            y.shape[0], _ptr(ws), ws.numel(), _stream(stream)), "lora_apply")
+
+
+def lora_apply_multi(pool: PoolHandle, targets, x, y, y_cols, ids, scales, ws, stream=None) -> None:
+    """Several same-shape targets sharing x in one call; target i adds its
+    delta to columns y_cols[i] .. y_cols[i] + d_out - 1 of y."""
+    n = len(targets)
+    t_arr = (ctypes.c_int * n)(*[int(t) for t in targets])
+    c_arr = (ctypes.c_int * n)(*[int(c) for c in y_cols])
+    _check(_lib.lora_apply_multi(pool, n, t_arr, _ptr(x), _ld(x), _ptr(y), _ld(y), c_arr, _ptr(ids), _ptr(scales),
+                                 y.shape[0], _ptr(ws), ws.numel(), _stream(stream)), "lora_apply_multi")
 
 
 def lora_apply_segments(pool: PoolHandle, target: int, x, y, seg_offsets, seg_slot, scales, ws,

@@ -140,6 +140,36 @@ int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ld
   return lora_apply_plan(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, stream);
 }
 
+int lora_apply_multi(lora_pool *p, int n_targets, const int *targets, const void *x, int ldx, void *y, int ldy,
+                     const int *y_cols, const int32_t *ids, const float *scales, int T, void *ws, size_t ws_bytes,
+                     void *stream) {
+  if (!p || !targets || !y_cols || n_targets < 1 || n_targets > kMaxMulti) return LORA_ERR_INVALID_ARG;
+  int rc = check_call(p, targets[0], T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  const int d_in = p->targets[targets[0]].d_in, d_out = p->targets[targets[0]].d_out;
+  for (int i = 0; i < n_targets; ++i) {
+    const int t = targets[i];
+    if (t < 0 || t >= p->n_targets) return LORA_ERR_INVALID_ARG;
+    if (p->targets[t].d_in != d_in || p->targets[t].d_out != d_out) return LORA_ERR_INVALID_ARG;
+    if (y_cols[i] < 0 || (long long)y_cols[i] + d_out > ldy) return LORA_ERR_INVALID_ARG;
+    if (y_cols[i] % 8) return LORA_ERR_ALIGNMENT;
+    for (int k = 0; k < i; ++k)  // the targets' column ranges must not overlap
+      if (y_cols[k] < y_cols[i] + d_out && y_cols[i] < y_cols[k] + d_out) return LORA_ERR_INVALID_ARG;
+  }
+  if ((rc = check_rows(x, ldx, d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, d_out)) != LORA_OK) return rc;
+  if (!scales || !ids) return LORA_ERR_INVALID_ARG;
+  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T <= kFusedMaxT) {
+    DeviceGuard g(p->device);
+    return launch_decode_multi(p, n_targets, targets, y_cols, x, ldx, y, ldy, scales, ids, T, nullptr, st);
+  }
+  if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
+  DeviceGuard g(p->device);
+  return launch_decode_multi(p, n_targets, targets, y_cols, x, ldx, y, ldy, scales, nullptr, T, ws, st);
+}
+
 int lora_apply_segments(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
                         const int32_t *seg_offsets, const int32_t *seg_slot, int S, const float *scales, int T,
                         void *ws, size_t ws_bytes, void *stream) {

@@ -36,6 +36,7 @@ constexpr int kClusterCtas = 8;      // CTAs that split one work item (portable 
 constexpr int kMaxStages = 4;        // pipeline depth of the decode kernel
 constexpr int kItemSlots = 8;        // items a warp's copies may run ahead of its compute
 constexpr int kFusedMaxT = 256;      // batches up to this size are grouped inside the decode kernel
+constexpr int kMaxMulti = 4;         // targets sharing x in one decode launch
 
 extern std::atomic<uint64_t> g_launches;
 
@@ -321,6 +322,12 @@ int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, in
 // kernel and no workspace.
 int launch_decode_ids(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
                       const float *scales, float *v, int ldv, const int32_t *ids, int T, cudaStream_t st);
+// Fused decode over n_tgt targets that share x (same d_in and d_out); target
+// i writes columns y_cols[i] .. + d_out - 1 of y.  ids != nullptr: grouped in
+// the kernel (T <= kFusedMaxT); else the plan in ws.
+int launch_decode_multi(lora_pool *pool, int n_tgt, const int *targets, const int *y_cols, const void *x, int ldx,
+                        void *y, int ldy, const float *scales, const int32_t *ids, int T, const void *ws,
+                        cudaStream_t st);
 struct PrefillGeometry {
   int r_cap, kb_per, n_ks, n_stages, n_groups, smem_sh, smem_ex;
 };

@@ -33,8 +33,13 @@ namespace lora {
 
 struct DecodeArgs {
   PoolView pool;
-  int target, d_in, d_out, r_max;
-  long long a_off, bt_off;
+  int d_in, d_out, r_max;
+  // targets of this launch: all share x, d_in and d_out; work unit u is
+  // (item u / n_tgt, target u % n_tgt); target i writes its delta into
+  // columns y_col[i] .. y_col[i] + d_out - 1 of y
+  int n_tgt;
+  int tgt[kMaxMulti];
+  long long a_off[kMaxMulti], bt_off[kMaxMulti], y_col[kMaxMulti];
   const uint16_t *x;
   long long ldx;
   uint16_t *y;
@@ -162,7 +167,8 @@ __device__ __forceinline__ void expand_prepare(const float *s_v, int r, int m, E
 template <int JB>
 __device__ __forceinline__ void expand_group(uint32_t buf_u, const uint8_t *yb, uint32_t zero_u, int pitch, int wv,
                                              int v_lo, int r, int m, const ExpandA<JB> &A, float scale,
-                                             const int *s_rows, const DecodeArgs &a, int lane, int cg) {
+                                             const int *s_rows, long long ycol, const DecodeArgs &a, int lane,
+                                             int cg) {
   const int g = lane >> 2, t = lane & 3;
   const int bj = (lane & 7) + ((lane >> 3) & 1) * 8, bn = (lane >> 4) * 16;
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -190,7 +196,7 @@ __device__ __forceinline__ void expand_group(uint32_t buf_u, const uint8_t *yb, 
         const uint32_t yv = *reinterpret_cast<const uint32_t *>(yb + i * pitch + col * 2);
         const uint32_t o = pack_bf16x2(fmaf(scale, acc[nt][2 * hr], bf16_lo(yv)),
                                        fmaf(scale, acc[nt][2 * hr + 1], bf16_hi(yv)));
-        *reinterpret_cast<uint32_t *>(a.y + (long long)s_rows[i] * a.ldy + (long long)v_lo * 8 + col) = o;
+        *reinterpret_cast<uint32_t *>(a.y + (long long)s_rows[i] * a.ldy + ycol + (long long)v_lo * 8 + col) = o;
       }
     }
   }
@@ -201,12 +207,14 @@ __device__ __forceinline__ void expand_group(uint32_t buf_u, const uint8_t *yb, 
 template <int JB>
 __device__ __forceinline__ void expand_mma(uint32_t buf_u, const uint8_t *yb, uint32_t zero_u, int pitch, int wv,
                                            int v_lo, int r, int m, const ExpandA<JB> &A, float scale,
-                                           const int *s_rows, const DecodeArgs &a, int lane, int warp) {
+                                           const int *s_rows, long long ycol, const DecodeArgs &a, int lane,
+                                           int warp) {
   const int groups = (wv + 1) / 2;  // 16-column groups (an odd last vector is half a group)
   for (int cg = warp; cg < groups; cg += 2 * kConsumerWarps) {
-    expand_group<JB>(buf_u, yb, zero_u, pitch, wv, v_lo, r, m, A, scale, s_rows, a, lane, cg);
+    expand_group<JB>(buf_u, yb, zero_u, pitch, wv, v_lo, r, m, A, scale, s_rows, ycol, a, lane, cg);
     if (cg + kConsumerWarps < groups)
-      expand_group<JB>(buf_u, yb, zero_u, pitch, wv, v_lo, r, m, A, scale, s_rows, a, lane, cg + kConsumerWarps);
+      expand_group<JB>(buf_u, yb, zero_u, pitch, wv, v_lo, r, m, A, scale, s_rows, ycol, a, lane,
+                       cg + kConsumerWarps);
   }
 }
 
@@ -281,7 +289,7 @@ __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;
 struct ItemInfo {
   int m, r;
   float scale;
-  int pad;
+  int ycol;  // first column of the unit's target in y
   int rows[kItemRows];
 };
 
@@ -362,7 +370,7 @@ __device__ int fused_plan(const DecodeArgs &a, const DecodeSmem &S, int tid, con
       } else {
         key = id;
         const PoolView &p = a.pool;
-        sinfo.x = p.rank[(long long)id * p.n_targets + a.target];
+        sinfo.x = p.rank[(long long)id * p.n_targets + a.tgt[0]];
         sinfo.y = slice_page(p, id, geo.a_first, geo.a_last);
         sinfo.z = slice_page(p, id, geo.b_first, geo.b_last);
         sinfo.w = a.scales ? __float_as_int(a.scales[id]) : 0;
@@ -429,6 +437,7 @@ struct IssueState {
   int li, tt;
   int slot, m, r;
   bool split_a, split_b;
+  long long a_off, bt_off;  // the unit's target blocks inside a slot
   unsigned long long wa0, wa1, wb0, wb1, xrow, yrow;
 };
 
@@ -468,50 +477,68 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   const int per_i = (nvi + C - 1) / C, per_o = (nvo + C - 1) / C;
   const int kv0 = min(crank * per_i, nvi), kv1 = min(kv0 + per_i, nvi);
   const int nv0 = min(crank * per_o, nvo), nv1 = min(nv0 + per_o, nvo);
-  // logical byte ranges of this CTA's A and B^T slices, rows 0 .. r_max-1
-  SliceGeo geo;
-  geo.a_first = geo.b_first = -1;
-  geo.a_last = geo.b_last = -1;
-  if (MODE != kExpandOnly && kv1 > kv0) {
-    geo.a_first = a.a_off + (long long)kv0 * 16;
-    geo.a_last = a.a_off + ((long long)(a.r_max - 1) * a.d_in + (long long)kv1 * 8) * 2 - 1;
-  }
-  if (MODE != kShrinkOnly && nv1 > nv0) {
-    geo.b_first = a.bt_off + (long long)nv0 * 16;
-    geo.b_last = a.bt_off + ((long long)(a.r_max - 1) * a.d_out + (long long)nv1 * 8) * 2 - 1;
-  }
+  // logical byte ranges of this CTA's A and B^T slices of target i, rows
+  // 0 .. r_max-1
+  auto slice_geo = [&](int i) {
+    SliceGeo g;
+    g.a_first = g.b_first = -1;
+    g.a_last = g.b_last = -1;
+    if (MODE != kExpandOnly && kv1 > kv0) {
+      g.a_first = a.a_off[i] + (long long)kv0 * 16;
+      g.a_last = a.a_off[i] + ((long long)(a.r_max - 1) * a.d_in + (long long)kv1 * 8) * 2 - 1;
+    }
+    if (MODE != kShrinkOnly && nv1 > nv0) {
+      g.b_first = a.bt_off[i] + (long long)nv0 * 16;
+      g.b_last = a.bt_off[i] + ((long long)(a.r_max - 1) * a.d_out + (long long)nv1 * 8) * 2 - 1;
+    }
+    return g;
+  };
+  // rank, scale and slice pages of a slot on target i, read from the tables
+  auto slot_info = [&](int slot, int i) {
+    const PoolView &p = a.pool;
+    const SliceGeo g = slice_geo(i);
+    return make_int4(p.rank[(long long)slot * p.n_targets + a.tgt[i]], slice_page(p, slot, g.a_first, g.a_last),
+                     slice_page(p, slot, g.b_first, g.b_last), a.scales ? __float_as_int(a.scales[slot]) : 0);
+  };
 
-  // ---- the item list, and this cluster's items resolved once: item k of
-  // the cluster (global index cid + k * ncl) gets its slot, rows, rank, scale
-  // and the physical pages of this CTA's slices, gathered by thread k.
-  // Grouped here from the index vector (all in shared memory), or read from
-  // the plan: its header and thread k's item record are read together (the
-  // items array has room for items_cap entries), then rank, scale and pages.
+  // ---- the item list, and this cluster's work units resolved once: unit k
+  // of the cluster (global unit cid + k * ncl = item * n_tgt + target) gets
+  // its slot, rows, rank, scale and the physical pages of this CTA's slices,
+  // gathered by thread k.  Grouped here from the index vector (for a single
+  // target all of it was gathered while grouping), or read from the plan:
+  // its header and thread k's item record are read together (the items array
+  // has room for items_cap entries), then rank, scale and pages.
   const bool fused = a.ids != nullptr;
+  const int NT = a.n_tgt;
   const int32_t *perm = a.perm;
   int n_items;
   int any_bad = 1;  // (plan path: the plan kernel reported empty slots itself)
   int4 rec = make_int4(0, 0, 0, 0), res = make_int4(-1, -1, 0, 0);
-  if (fused) {
-    n_items = fused_plan(a, S, tid, geo, &any_bad);
-    perm = S.f_perm;
-    const int k = cid + tid * ncl;
-    if (k < n_items) {
-      rec = unpack_item(S.f_items[k]);
-      const int4 sl = S.f_slot[rec.y];
-      rec.w = sl.x;
-      res = make_int4(sl.y, sl.z, sl.w, 0);
-    }
-  } else {
-    const int k = cid + tid * ncl;
-    int4 d = make_int4(0, 0, 0, 0);
-    if (k < a.items_cap) d = a.items[k];
-    n_items = a.hdr[a.items_hdr];
-    if (k < n_items) {
-      const PoolView &p = a.pool;
-      rec = make_int4(d.x, d.y, d.z, p.rank[(long long)d.x * p.n_targets + a.target]);
-      res = make_int4(slice_page(p, d.x, geo.a_first, geo.a_last), slice_page(p, d.x, geo.b_first, geo.b_last),
-                      a.scales ? __float_as_int(a.scales[d.x]) : 0, 0);
+  {
+    const int u = cid + tid * ncl, item = u / NT, ti = u - item * NT;
+    if (fused) {
+      n_items = fused_plan(a, S, tid, slice_geo(0), &any_bad);
+      perm = S.f_perm;
+      if (item < n_items) {
+        rec = unpack_item(S.f_items[item]);
+        int4 sl;
+        if (NT == 1) {
+          sl = S.f_slot[rec.y];
+        } else {
+          sl = slot_info(rec.x, ti);
+        }
+        rec.w = sl.x;
+        res = make_int4(sl.y, sl.z, sl.w, ti);
+      }
+    } else {
+      int4 d = make_int4(0, 0, 0, 0);
+      if (item < a.items_cap) d = a.items[item];
+      n_items = a.hdr[a.items_hdr];
+      if (item < n_items) {
+        const int4 sl = slot_info(d.x, ti);
+        rec = make_int4(d.x, d.y, d.z, sl.x);
+        res = make_int4(sl.y, sl.z, sl.w, ti);
+      }
     }
   }
   __syncthreads();  // (the grouping's arrays are read before they are reused)
@@ -521,7 +548,8 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   const int nk = (MODE == kExpandOnly) ? 0 : (per_i + TV - 1) / TV;
   const int nn = (MODE == kShrinkOnly) ? 0 : (per_o + TV - 1) / TV;
   const int tpi = nk + nn;
-  const int my_items = cid < n_items ? (n_items - cid + ncl - 1) / ncl : 0;
+  const int n_units = n_items * NT;
+  const int my_items = cid < n_units ? (n_units - cid + ncl - 1) / ncl : 0;  // this cluster's units
   const int total = my_items * tpi;
   const int wlen_a = (kv1 - kv0) * 16, wlen_b = (nv1 - nv0) * 16;
 
@@ -534,17 +562,20 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
   is.tt = 0;
   auto resolve = [&](int li) {
     int4 d, sinfo;
+    int ti;
     if (li < kDecodeThreads) {
       d = S.it_rec[li];
       const int4 rs = S.it_res[li];
       sinfo = make_int4(d.w, rs.x, rs.y, rs.z);
+      ti = rs.w;
     } else {
-      d = a.items[cid + li * ncl];
-      sinfo = make_int4(a.pool.rank[(long long)d.x * a.pool.n_targets + a.target],
-                        slice_page(a.pool, d.x, geo.a_first, geo.a_last),
-                        slice_page(a.pool, d.x, geo.b_first, geo.b_last),
-                        a.scales ? __float_as_int(a.scales[d.x]) : 0);
+      const int u = cid + li * ncl, item = u / NT;
+      ti = u - item * NT;
+      d = fused ? unpack_item(S.f_items[item]) : a.items[item];
+      sinfo = slot_info(d.x, ti);
     }
+    is.a_off = a.a_off[ti];
+    is.bt_off = a.bt_off[ti];
     is.slot = d.x;
     is.m = d.z;
     const float scale = __int_as_float(sinfo.w);
@@ -557,7 +588,7 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
       if (j < a.r_max) {
         long long room;
         if (MODE != kExpandOnly && wlen_a > 0) {
-          const long long off = a.a_off + ((long long)j * a.d_in + (long long)kv0 * 8) * 2;
+          const long long off = is.a_off + ((long long)j * a.d_in + (long long)kv0 * 8) * 2;
           if (sinfo.y >= 0) {
             wa[h] = a.pool.base + (long long)sinfo.y * a.pool.page_bytes +
                     (a.pool.log2_page < 0 ? off : off & (a.pool.page_bytes - 1));
@@ -567,7 +598,7 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
           }
         }
         if (MODE != kShrinkOnly && wlen_b > 0) {
-          const long long off = a.bt_off + ((long long)j * a.d_out + (long long)nv0 * 8) * 2;
+          const long long off = is.bt_off + ((long long)j * a.d_out + (long long)nv0 * 8) * 2;
           if (sinfo.z >= 0) {
             wb[h] = a.pool.base + (long long)sinfo.z * a.pool.page_bytes +
                     (a.pool.log2_page < 0 ? off : off & (a.pool.page_bytes - 1));
@@ -588,13 +619,14 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
     is.wb0 = (unsigned long long)wb[0];
     is.wb1 = (unsigned long long)wb[1];
     is.xrow = a.x ? (unsigned long long)(a.x + (long long)my_row * a.ldx + (long long)kv0 * 8) : 0ull;
-    is.yrow = a.y ? (unsigned long long)(a.y + (long long)my_row * a.ldy + (long long)nv0 * 8) : 0ull;
+    is.yrow = a.y ? (unsigned long long)(a.y + (long long)my_row * a.ldy + a.y_col[ti] + (long long)nv0 * 8) : 0ull;
     ItemInfo &I = my_info[li % kItemSlots];
     if (lane < is.m) I.rows[lane] = my_row;
     if (lane == 0) {
       I.m = is.m;
       I.r = is.r;
       I.scale = scale;
+      I.ycol = (int)a.y_col[ti];
     }
     __syncwarp();
   };
@@ -628,7 +660,7 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
       if (q < is.r) {
         const long long off = (long long)t_idx * TV * 16;
         if (split) {  // the slice crosses a page: copy it piece by piece
-          const long long loff = (shrink ? a.a_off + (long long)q * a.d_in * 2 : a.bt_off + (long long)q * a.d_out * 2) +
+          const long long loff = (shrink ? is.a_off + (long long)q * a.d_in * 2 : is.bt_off + (long long)q * a.d_out * 2) +
                                  (long long)v_lo * 16;
           copy_pool_row(a.pool, is.slot, loff, bytes, buf + q * pitch, &S.full[stage], a.status);
         } else {
@@ -723,8 +755,8 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
       } else {
         if (t_idx == 0) expand_prepare<JB>(S.v, r, m, va, lane);
         if (wv > 0)
-          expand_mma<JB>(buf_u, buf + act_base, smem_u32(S.zero), pitch, wv, v_lo, r, m, va, scale, I.rows, a, lane,
-                         warp);
+          expand_mma<JB>(buf_u, buf + act_base, smem_u32(S.zero), pitch, wv, v_lo, r, m, va, scale, I.rows, I.ycol, a,
+                         lane, warp);
       }
     }
     __syncwarp();
@@ -884,17 +916,22 @@ int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx,
   return launch_decode_items(pool, mode, target, x, ldx, y, ldy, scales, v, ldv, T, ws, st, kHdrItems);
 }
 
-static int launch_decode_args(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
-                              const float *scales, float *v, int ldv, int T, const void *ws, const int32_t *ids,
-                              cudaStream_t st, int items_hdr) {
+static int launch_decode_args(lora_pool *pool, int mode, int n_tgt, const int *targets, const int *y_cols,
+                              const void *x, int ldx, void *y, int ldy, const float *scales, float *v, int ldv,
+                              int T, const void *ws, const int32_t *ids, cudaStream_t st, int items_hdr) {
   DecodeArgs a;
   a.pool = pool->view();
-  a.target = target;
-  a.d_in = pool->targets[target].d_in;
-  a.d_out = pool->targets[target].d_out;
+  a.d_in = pool->targets[targets[0]].d_in;
+  a.d_out = pool->targets[targets[0]].d_out;
   a.r_max = pool->r_max;
-  a.a_off = pool->a_off[target];
-  a.bt_off = pool->bt_off[target];
+  a.n_tgt = n_tgt;
+  for (int i = 0; i < kMaxMulti; ++i) {
+    const int t = targets[i < n_tgt ? i : 0];
+    a.tgt[i] = t;
+    a.a_off[i] = pool->a_off[t];
+    a.bt_off[i] = pool->bt_off[t];
+    a.y_col[i] = (y_cols && i < n_tgt) ? y_cols[i] : 0;
+  }
   a.x = static_cast<const uint16_t *>(x);
   a.ldx = ldx;
   a.y = static_cast<uint16_t *>(y);
@@ -924,14 +961,19 @@ static int launch_decode_args(lora_pool *pool, int mode, int target, const void 
   a.n_stages = ns;
   decode_geometry(pool->r_max, &a.tile_vecs, &a.row_pitch, &ns);
   // Items are bounded by min(T, n_slots) segments plus T / kItemRows chunk
-  // splits; clusters loop over items, so the grid never exceeds what fits.
+  // splits (times the targets: one work unit per item and target); clusters
+  // loop over units, so the grid never exceeds what fits.
   // A batch that may hold more than twice as many items as there are 8-CTA
   // clusters takes 4-CTA clusters: twice the items in flight, each split
   // four ways instead of eight.  (Up to rank 32 only: with rank 64 the
   // 512-byte rows double the tiles of each item and it measured slower.)
-  const long long bound = (long long)std::min(T, pool->n_slots) + (T + kItemRows - 1) / kItemRows;
+  // (The cluster size follows the items of one target, so that a launch over
+  // several targets splits each item exactly as a launch per target would:
+  // measured, the finer split gave a launch over q, k and v no gain.)
+  const long long items1 = (long long)std::min(T, pool->n_slots) + (T + kItemRows - 1) / kItemRows;
+  const long long bound = items1 * (long long)n_tgt;
   const bool small_clusters =
-      pool->r_max <= 32 && bound > 2LL * pool->decode_max_clusters && pool->decode_max_clusters4 > 0;
+      pool->r_max <= 32 && items1 > 2LL * pool->decode_max_clusters && pool->decode_max_clusters4 > 0;
   const int csize = small_clusters ? kClusterCtas / 2 : kClusterCtas;
   int n_clusters = (int)std::min<long long>(
       bound, (long long)(small_clusters ? pool->decode_max_clusters4 : pool->decode_max_clusters));
@@ -952,13 +994,23 @@ static int launch_decode_args(lora_pool *pool, int mode, int target, const void 
 int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
                         const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
                         int items_hdr) {
-  return launch_decode_args(pool, mode, target, x, ldx, y, ldy, scales, v, ldv, T, ws, nullptr, st, items_hdr);
+  return launch_decode_args(pool, mode, 1, &target, nullptr, x, ldx, y, ldy, scales, v, ldv, T, ws, nullptr, st,
+                            items_hdr);
 }
 
 int launch_decode_ids(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
                       const float *scales, float *v, int ldv, const int32_t *ids, int T, cudaStream_t st) {
   if (T < 1 || T > kFusedMaxT) return LORA_ERR_INVALID_ARG;
-  return launch_decode_args(pool, mode, target, x, ldx, y, ldy, scales, v, ldv, T, nullptr, ids, st, kHdrItems);
+  return launch_decode_args(pool, mode, 1, &target, nullptr, x, ldx, y, ldy, scales, v, ldv, T, nullptr, ids, st,
+                            kHdrItems);
+}
+
+int launch_decode_multi(lora_pool *pool, int n_tgt, const int *targets, const int *y_cols, const void *x, int ldx,
+                        void *y, int ldy, const float *scales, const int32_t *ids, int T, const void *ws,
+                        cudaStream_t st) {
+  if (n_tgt < 1 || n_tgt > kMaxMulti || (ids && (T < 1 || T > kFusedMaxT))) return LORA_ERR_INVALID_ARG;
+  return launch_decode_args(pool, kFused, n_tgt, targets, y_cols, x, ldx, y, ldy, scales, nullptr, 0, T, ws, ids,
+                            st, kHdrItems);
 }
 
 }  // namespace lora

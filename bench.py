@@ -1,7 +1,7 @@
 """Benchmark of the multi-LoRA delta path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload q_proj|tiny|prefill|mlp|paged]
+                    [--workload q_proj|tiny|prefill|mlp|paged|qkv]
 
 Default workload (the metric's configuration): Llama-2-7B q_proj-shaped decode,
 d_in = d_out = 4096, rank 16 for all, 32 resident adapters in a contiguous
@@ -43,7 +43,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "LoRA-delta tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
-WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5}
+WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5, "qkv": 2}
 L2_BYTES = 126 * 2 ** 20
 FUSED_MAX_T = 256   # batches up to this size are grouped inside the decode kernel (one launch)
 
@@ -179,7 +179,7 @@ def run_reference(args, rank: int, world: int):
         return
     import synth
     w = synth.config(WORKLOADS[args.workload])
-    n_t = len(w.targets) if args.workload == "paged" else 1
+    n_t = len(w.targets) if args.workload == "paged" else 3 if args.workload == "qkv" else 1
     threads = min(cpu_threads(), w.T)
     inp = oracle_inputs(w, 0)
     time_oracle(w, inp, 0.0, threads, max_calls=args.warmup)
@@ -235,6 +235,8 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     scales = torch.from_numpy(scales_np).to(dev)
     if args.workload == "paged":
         return run_paged(args, rank, world, dev, w, scales, bf16)
+    if args.workload == "qkv":
+        return run_qkv(args, rank, world, dev, w, scales, bf16)
 
     # one buffer set: pool (all slots loaded), x, y, ids, workspace
     pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
@@ -524,6 +526,105 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
                      "algorithmic_bytes_per_launch": alg},
         "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, n_t, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def run_qkv(args, rank, world, dev, w2, scales, bf16):
+    """The q_proj decode batch (64 tokens, 32 rank-16 adapters, ids of the
+    q_proj workload) on the q, k and v projections of one layer (three
+    4096 x 4096 targets with their own adapter weights) that share x: one
+    lora_apply_multi per step into a fused [64, 3 x 4096] y, against three
+    lora_apply calls for context."""
+    import torch
+
+    import adapter_deltas_b200 as L
+    import synth
+    d = 4096
+    w = synth.custom(2000 + rank, w2.T, [(d, d)] * 3, [int(r) for r in w2.rank], int(w2.r_max), ids=w2.ids)
+    T, n_t = w.T, 3
+    cols = [0, d, 2 * d]
+    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, 0)
+    act_bytes = T * (d + 3 * d) * 2
+    n_sets = max(2, min(64, -(-4 * L2_BYTES // (pool_bytes + act_bytes))))
+    adapters = {}
+    for s_ in range(w.n_slots):
+        for t in range(n_t):
+            A, B = w.adapter(s_, t)
+            adapters[(s_, t)] = (bf16(A), bf16(B))
+    x0 = bf16(w.x(0))
+    y0 = torch.cat([bf16(w.y_in(t)) for t in range(n_t)], dim=1).contiguous()
+    ids0 = torch.from_numpy(w.ids).to(dev)
+    sets = []
+    for k in range(n_sets):
+        mem = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
+        pool = L.lora_pool_create(dev.index, w.targets, w.r_max, w.n_slots, 0, mem, 0)
+        for (s_, t), (A, B) in adapters.items():
+            L.lora_pool_load(pool, s_, t, int(w.rank[s_]), A, B)
+        ws = torch.zeros(L.lora_workspace_bytes(pool, 0, T), dtype=torch.uint8, device=dev)
+        sets.append(dict(pool=pool, mem=mem, x=x0.clone(), y=y0.clone(), ids=ids0.clone(), ws=ws))
+    torch.cuda.synchronize()
+
+    def step(k):
+        s_ = sets[k % n_sets]
+        L.lora_apply_multi(s_["pool"], [0, 1, 2], s_["x"], s_["y"], cols, s_["ids"], scales, s_["ws"])
+
+    def step_separate(k):
+        s_ = sets[k % n_sets]
+        for t in range(n_t):
+            L.lora_apply(s_["pool"], t, s_["x"], s_["y"][:, cols[t]:cols[t] + d], s_["ids"], scales, s_["ws"])
+
+    def timed(fn, n):
+        g_w, _ = capture_graph(dev, fn, range(args.warmup))
+        g, launches = capture_graph(dev, fn, range(n))
+        g_w.replay()
+        torch.cuda.synchronize()
+        sync_ranks(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        g.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        sync_ranks(world)
+        return ev0.elapsed_time(ev1) / n, launches, (g, g_w)
+
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        ms, launches, keep = timed(step, args.steps)
+    clocks = sampler.stop()
+    ms = reduce_max(ms, world, dev)
+    sep_ms, _, keep2 = timed(step_separate, args.steps)
+    sep_ms = reduce_max(sep_ms, world, dev)
+    del keep, keep2
+    for s_ in sets:
+        L.lora_pool_destroy(s_["pool"])
+    if rank != 0:
+        return
+    peak, peak_kind = load_peaks()
+    # algorithmic bytes: each distinct adapter's A and B on the three targets,
+    # x of the adapted rows once (shared), y of the adapted rows read and
+    # written on each target
+    act = w.ids[w.ids >= 0]
+    distinct = np.unique(act)
+    alg = int(sum(int(w.rank[a]) * 2 * d * 2 for a in distinct)) * n_t + act.size * d * 2 + n_t * act.size * d * 4
+    achieved = alg / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": job_value(T, world, ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "qkv decode: q_proj batch on 3 targets sharing x, d4096 r16 32 adapters 64 tokens",
+                   "global_batch": T * world, "seq_len": 1,
+                   "parallelism": "replicas%d" % world if world > 1 else "single", "deltas_per_step": n_t,
+                   "l2": "%d rotating buffer sets > 4x L2" % n_sets,
+                   "timing": "CUDA graph of the K steps, CUDA events around its replay"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": None, "kernel": "decode_kernel<fused>, 3 targets per launch",
+                     "kernel_us": ms * 1e3, "algorithmic_bytes_per_launch": alg},
+        "separate_launches": {"ms_per_step": sep_ms, "value": job_value(T, world, sep_ms),
+                              "note": "the same three deltas as three lora_apply calls"},
         "gpu_launches": launches, "clocks": clocks,
     }
     if world == 1:

@@ -263,6 +263,34 @@ LORA_API int lora_apply(lora_pool *pool, int target, const void *x, int ldx, voi
                int ldy, const int32_t *ids, const float *scales, int T,
                void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Several targets that read the same x -- the q, k and v projections of one
+ * layer (the target modules of "Multi-LoRA Serving: Why 100 Adapters Fit on
+ * One GPU", section "How much memory does one LoRA adapter actually cost?")
+ * -- in one launch: for i < n_targets,
+ *     y[t, y_cols[i] + n] += scales[a] * (B_a (A_a x[t]))[n],  a = ids[t],
+ * with A_a, B_a the adapter's matrices on target targets[i].  Equal to
+ * n_targets lora_apply calls on the column slices of y, bit for bit.
+ *   n_targets  1 .. 4
+ *   targets    host int [n_targets]: target indices, all with the same d_in
+ *              and the same d_out
+ *   y_cols     host int [n_targets]: first column of each target's slice of
+ *              y, a multiple of 8; slices may not overlap and must end within
+ *              ldy (e.g. 0, d_out, 2 d_out for a fused qkv output)
+ *   x, ldx     device bf16 [T, ldx], shared by all the targets
+ *   y, ldy     device bf16 [T, ldy], updated in place
+ *   ids, scales, T, ws, ws_bytes, stream  as for lora_apply (ws sized for
+ *              targets[0]); batches of at most 256 rows take one launch and
+ *              leave ws unwritten.
+ * Errors: LORA_ERR_INVALID_ARG for a bad count, target, shape mismatch,
+ * overlapping or out-of-range slice; LORA_ERR_ALIGNMENT for a column not a
+ * multiple of 8; device-side statuses as for lora_apply.
+ */
+LORA_API int lora_apply_multi(lora_pool *pool, int n_targets, const int *targets,
+                     const void *x, int ldx, void *y, int ldy, const int *y_cols,
+                     const int32_t *ids, const float *scales, int T, void *ws,
+                     size_t ws_bytes, void *stream);
+
 /* lora_plan_segments followed by lora_apply_plan. */
 LORA_API int lora_apply_segments(lora_pool *pool, int target, const void *x, int ldx,
                         void *y, int ldy, const int32_t *seg_offsets,
