@@ -70,6 +70,9 @@ _sig("lora_pool_bytes_required", _Z, [_P, _I, _I, _I, _Z])
 _sig("lora_pool_create", _I, [ctypes.POINTER(_P), _I, _P, _I, _I, _I, _Z, _P, _Z, ctypes.c_uint64])
 _sig("lora_pool_load", _I, [_P, _I, _I, _I, _P, _P, _I, _P])
 _sig("lora_pool_unload", _I, [_P, _I])
+_sig("lora_pool_swap_in", _I, [_P, _I, _P, _P, _Z, _P, _Z, _P])
+_sig("lora_swap_src_bytes", _Z, [_P, _P])
+_sig("lora_swap_staging_bytes", _Z, [_P, _P])
 _sig("lora_pool_destroy", _I, [_P])
 _sig("lora_pool_page_table", _P, [_P])
 _sig("lora_pool_get_info", _I, [_P, ctypes.POINTER(lora_pool_info)])
@@ -176,6 +179,27 @@ def lora_pool_load(pool: PoolHandle, slot: int, target: int, rank: int, A, B, st
         assert A.is_contiguous() and B.is_contiguous()
     _check(_lib.lora_pool_load(pool, slot, target, rank, _ptr(A), _ptr(B), on_dev, _stream(stream)),
            "lora_pool_load")
+
+
+def _int_array(values):
+    values = [int(v) for v in values]
+    return (ctypes.c_int * len(values))(*values)
+
+
+def lora_swap_src_bytes(pool: PoolHandle, ranks) -> int:
+    return int(_lib.lora_swap_src_bytes(pool, _int_array(ranks)))
+
+
+def lora_swap_staging_bytes(pool: PoolHandle, ranks) -> int:
+    return int(_lib.lora_swap_staging_bytes(pool, _int_array(ranks)))
+
+
+def lora_pool_swap_in(pool: PoolHandle, slot: int, ranks, src, staging, stream=None) -> None:
+    """One adapter, all targets, from host memory `src` (a CPU tensor, pinned
+    for an asynchronous copy) through the device tensor `staging`."""
+    nbytes = src.numel() * src.element_size()
+    _check(_lib.lora_pool_swap_in(pool, slot, _int_array(ranks), _ptr(src), nbytes, _ptr(staging),
+                                  staging.numel() * staging.element_size(), _stream(stream)), "lora_pool_swap_in")
 
 
 def lora_pool_unload(pool: PoolHandle, slot: int) -> None:

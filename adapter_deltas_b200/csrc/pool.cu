@@ -92,9 +92,71 @@ __global__ void store_bt_kernel(PoolView pool, int slot, long long bt_off, int d
   *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(dst)) = packed;
 }
 
+// One target's part of a swap-in: where its A (then its B) sits in the
+// staging data and where the target's blocks lie in a slot.
+struct SwapDesc {
+  long long src, a_off, bt_off, pad;
+  int d_in, d_out, rank, pad2;
+};
+static_assert(sizeof(SwapDesc) == 48, "descriptor layout");
+
+// Staged adapter -> one slot's pages: block y handles target y; its threads
+// walk the target's A block (r_max x d_in) then its B^T block (r_max x d_out)
+// in 16-byte chunks -- rows below the rank from the staged A and (transposed)
+// B, the padding rows as zeros -- and store each through the page table.
+__global__ void swap_in_kernel(PoolView pool, int slot, int r_max, const SwapDesc *desc, const uint8_t *data) {
+  const SwapDesc d = desc[blockIdx.y];
+  const long long per_a = d.d_in / 8, per_b = d.d_out / 8;
+  const long long na = (long long)r_max * per_a, nb = (long long)r_max * per_b;
+  const uint16_t *B = reinterpret_cast<const uint16_t *>(data + d.src + (long long)d.rank * d.d_in * 2);
+  for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < na + nb;
+       c += (long long)gridDim.x * blockDim.x) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    long long off;
+    if (c < na) {
+      const int j = (int)(c / per_a);
+      off = d.a_off + c * 16;
+      if (j < d.rank) v = *reinterpret_cast<const uint4 *>(data + d.src + c * 16);
+    } else {
+      const long long cb = c - na;
+      const int j = (int)(cb / per_b), n0 = (int)(cb % per_b) * 8;
+      off = d.bt_off + cb * 16;
+      if (j < d.rank) {
+        uint16_t e[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) e[q] = B[(long long)(n0 + q) * d.rank + j];
+        v.x = e[0] | (uint32_t(e[1]) << 16);
+        v.y = e[2] | (uint32_t(e[3]) << 16);
+        v.z = e[4] | (uint32_t(e[5]) << 16);
+        v.w = e[6] | (uint32_t(e[7]) << 16);
+      }
+    }
+    long long room;
+    const uint8_t *dst = pool_addr(pool, slot, off, &room);
+    if (dst) *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(dst)) = v;
+  }
+}
+
 }  // namespace lora
 
 using namespace lora;
+
+namespace {
+
+// Bytes of a packed swap-in source: for each target with rank > 0, A [rank,
+// d_in] then B [d_out, rank], bf16.  -1 for an invalid rank.
+long long swap_src_bytes(const lora_pool *p, const int *ranks) {
+  long long n = 0;
+  for (int t = 0; t < p->n_targets; ++t) {
+    if (ranks[t] < 0 || ranks[t] > p->r_max) return -1;
+    n += (long long)ranks[t] * (p->targets[t].d_in + p->targets[t].d_out) * 2;
+  }
+  return n;
+}
+
+size_t swap_desc_bytes(const lora_pool *p) { return align256(size_t(p->n_targets) * sizeof(SwapDesc)); }
+
+}  // namespace
 
 #define CUDA_TRY(expr)                            \
   do {                                            \
@@ -280,6 +342,74 @@ int lora_pool_load(lora_pool *p, int slot, int target, int rank, const void *A, 
                            p->rank.data() + (size_t)slot * p->n_targets + target, 4,
                            cudaMemcpyHostToDevice, st));
   if (!src_is_device) CUDA_TRY(cudaStreamSynchronize(st));  // host staging buffers go out of scope
+  return LORA_OK;
+}
+
+size_t lora_swap_src_bytes(const lora_pool *p, const int *ranks) {
+  if (!p || !ranks) return 0;
+  const long long n = swap_src_bytes(p, ranks);
+  return n < 0 ? 0 : size_t(n);
+}
+
+size_t lora_swap_staging_bytes(const lora_pool *p, const int *ranks) {
+  if (!p || !ranks) return 0;
+  const long long n = swap_src_bytes(p, ranks);
+  return n < 0 ? 0 : swap_desc_bytes(p) + size_t(n);
+}
+
+int lora_pool_swap_in(lora_pool *p, int slot, const int *ranks, const void *src, size_t src_bytes, void *staging,
+                      size_t staging_bytes, void *stream) {
+  if (!p || !ranks) return LORA_ERR_INVALID_ARG;
+  if (slot < 0 || slot >= p->n_slots) return LORA_ERR_SLOT;
+  const long long need = swap_src_bytes(p, ranks);
+  if (need < 0 || (long long)src_bytes != need) return LORA_ERR_INVALID_ARG;
+  if (need > 0 && !src) return LORA_ERR_INVALID_ARG;
+  if (!staging) return LORA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(staging) & 255u) return LORA_ERR_ALIGNMENT;
+  if (staging_bytes < swap_desc_bytes(p) + size_t(need)) return LORA_ERR_WORKSPACE;
+  std::lock_guard<std::mutex> lk(p->mu);
+  DeviceGuard g(p->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!p->loaded[slot]) {
+    if ((int)p->free_pages.size() < p->pps) return LORA_ERR_NO_PAGES;
+    for (int i = 0; i < p->pps; ++i) {
+      p->pt[(size_t)slot * p->pps + i] = p->free_pages.back();
+      p->free_pages.pop_back();
+    }
+    p->loaded[slot] = 1;
+    CUDA_TRY(cudaMemcpyAsync(p->d_pt + (size_t)slot * p->pps, p->pt.data() + (size_t)slot * p->pps,
+                             (size_t)p->pps * 4, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(p->d_loaded + slot, p->loaded.data() + slot, 4, cudaMemcpyHostToDevice, st));
+  }
+  // descriptors (a small pageable copy, staged by the driver before the call
+  // returns), then the adapter itself in one copy, then one scatter kernel
+  std::vector<SwapDesc> desc(p->n_targets);
+  long long off = 0, widest = 0;
+  for (int t = 0; t < p->n_targets; ++t) {
+    SwapDesc &d = desc[t];
+    d.src = off;
+    d.a_off = p->a_off[t];
+    d.bt_off = p->bt_off[t];
+    d.pad = 0;
+    d.d_in = p->targets[t].d_in;
+    d.d_out = p->targets[t].d_out;
+    d.rank = ranks[t];
+    d.pad2 = 0;
+    off += (long long)ranks[t] * (d.d_in + d.d_out) * 2;
+    widest = std::max(widest, (long long)p->r_max * (d.d_in + d.d_out) / 8);
+  }
+  uint8_t *stg = static_cast<uint8_t *>(staging);
+  CUDA_TRY(cudaMemcpyAsync(stg, desc.data(), desc.size() * sizeof(SwapDesc), cudaMemcpyHostToDevice, st));
+  if (need > 0) CUDA_TRY(cudaMemcpyAsync(stg + swap_desc_bytes(p), src, (size_t)need, cudaMemcpyHostToDevice, st));
+  const int threads = 256;
+  const unsigned bx = (unsigned)std::min<long long>(64, (widest + threads - 1) / threads);
+  g_launches.fetch_add(1);
+  swap_in_kernel<<<dim3(bx, (unsigned)p->n_targets), threads, 0, st>>>(
+      p->view(), slot, p->r_max, reinterpret_cast<const SwapDesc *>(stg), stg + swap_desc_bytes(p));
+  CUDA_TRY(cudaGetLastError());
+  for (int t = 0; t < p->n_targets; ++t) p->rank[(size_t)slot * p->n_targets + t] = ranks[t];
+  CUDA_TRY(cudaMemcpyAsync(p->d_rank + (size_t)slot * p->n_targets, p->rank.data() + (size_t)slot * p->n_targets,
+                           (size_t)p->n_targets * 4, cudaMemcpyHostToDevice, st));
   return LORA_OK;
 }
 

@@ -1,7 +1,7 @@
 """Benchmark of the multi-LoRA delta path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload q_proj|tiny|prefill|mlp|paged|qkv]
+                    [--workload q_proj|tiny|prefill|mlp|paged|qkv|swapin]
 
 Default workload (the metric's configuration): Llama-2-7B q_proj-shaped decode,
 d_in = d_out = 4096, rank 16 for all, 32 resident adapters in a contiguous
@@ -43,7 +43,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "LoRA-delta tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
-WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5, "qkv": 2}
+WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5, "qkv": 2, "swapin": 5}
 L2_BYTES = 126 * 2 ** 20
 FUSED_MAX_T = 256   # batches up to this size are grouped inside the decode kernel (one launch)
 
@@ -237,6 +237,8 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         return run_paged(args, rank, world, dev, w, scales, bf16)
     if args.workload == "qkv":
         return run_qkv(args, rank, world, dev, w, scales, bf16)
+    if args.workload == "swapin":
+        return run_swapin(args, rank, world, dev, bf16)
 
     # one buffer set: pool (all slots loaded), x, y, ids, workspace
     pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
@@ -629,6 +631,123 @@ def run_qkv(args, rank, world, dev, w2, scales, bf16):
     }
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(w, n_t, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def run_swapin(args, rank, world, dev, bf16):
+    """Adapter swap-in at the paged workload's geometry: one rank-16 adapter on
+    the q/k/v/o of 32 layers (128 targets of 4096 x 4096, 32 MiB) from pinned
+    host memory into 1 MiB pages, K swaps per measurement.  Reported against a
+    plain pinned host-to-device copy of the same bytes timed in the same run
+    (the link's measured rate), and against q_proj-shaped decode steps on
+    other slots run alone and beside the swap-ins on a second stream."""
+    import torch
+
+    import adapter_deltas_b200 as L
+    import synth
+    d, n_t, r, n_swap, n_res = 4096, 128, 16, 8, 4
+    ids = synth.config(2).ids % n_res + n_swap      # decode batch over the resident slots
+    w = synth.custom(3000 + rank, len(ids), [(d, d)] * n_t, [r] * (n_swap + n_res), r, ids=ids,
+                     page_bytes=1 << 20, scatter_seed=5)
+    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
+    mem = torch.zeros(pool_bytes, dtype=torch.uint8, device=dev)
+    pool = L.lora_pool_create(dev.index, w.targets, w.r_max, w.n_slots, w.page_bytes, mem, w.scatter_seed)
+    ranks = [r] * n_t
+    # one packed adapter (slot 0's weights) in pinned memory
+    parts = []
+    for t in range(n_t):
+        A, B = w.adapter(0, t)
+        parts += [np.ascontiguousarray(A).ravel(), np.ascontiguousarray(B).ravel()]
+    flat = np.concatenate(parts)
+    src = torch.empty(flat.size * 2, dtype=torch.uint8).pin_memory()
+    src.numpy()[:] = flat.view(np.uint8)
+    nbytes = src.numel()
+    staging = torch.empty(L.lora_swap_staging_bytes(pool, ranks), dtype=torch.uint8, device=dev)
+    plain_dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    for s_ in range(n_swap, n_swap + n_res):           # resident slots for the decode steps
+        L.lora_pool_swap_in(pool, s_, ranks, src, staging)
+    torch.cuda.synchronize()
+    s_swap, s_dec = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x = bf16(w.x(0))
+    y = bf16(w.y_in(0))
+    d_ids = torch.from_numpy(w.ids).to(dev)
+    sc = torch.full((w.n_slots,), 2.0, dtype=torch.float32, device=dev)
+    ws = torch.zeros(L.lora_workspace_bytes(pool, 0, w.T), dtype=torch.uint8, device=dev)
+
+    def swaps():
+        for k in range(n_swap):
+            L.lora_pool_swap_in(pool, k, ranks, src, staging, s_swap)
+
+    def plain():
+        for k in range(n_swap):
+            plain_dst.copy_(src, non_blocking=True)
+
+    def decode_steps(n):
+        with torch.cuda.stream(s_dec):
+            for k in range(n):
+                L.lora_apply(pool, k % 4, x, y, d_ids, sc, ws)
+
+    def timed(stream, fn):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    n_dec = 400
+    for _ in range(max(1, args.warmup)):
+        timed(s_swap, swaps)
+        timed(s_swap, plain)
+        timed(s_dec, lambda: decode_steps(n_dec))
+    launches0 = L.lora_kernel_launches()
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        swap_ms = min(timed(s_swap, swaps) for _ in range(args.steps))
+        plain_ms = min(timed(s_swap, plain) for _ in range(args.steps))
+        dec_ms = min(timed(s_dec, lambda: decode_steps(n_dec)) for _ in range(args.steps))
+        # both at once: decode steps on one stream, swap-ins on the other
+        both = []
+        for _ in range(args.steps):
+            torch.cuda.synchronize()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(s_dec)
+            e[2].record(s_swap)
+            decode_steps(n_dec)
+            with torch.cuda.stream(s_swap):
+                swaps()
+            e[1].record(s_dec)
+            e[3].record(s_swap)
+            torch.cuda.synchronize()
+            both.append((e[0].elapsed_time(e[1]), e[2].elapsed_time(e[3])))
+    clocks = sampler.stop()
+    launches = (L.lora_kernel_launches() - launches0) // max(1, args.steps)
+    L.lora_pool_destroy(pool)
+    if rank != 0:
+        return
+    dec_both = min(b[0] for b in both)
+    swap_both = min(b[1] for b in both)
+    gbs = n_swap * nbytes / (swap_ms * 1e-3) / 1e9
+    plain_gbs = n_swap * nbytes / (plain_ms * 1e-3) / 1e9
+    line = {
+        "metric": "adapter swap-in GB/s, pinned host to paged pool, 1 GPU", "value": gbs, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": swap_ms / n_swap,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "swap-in of one rank-16 adapter on 128 targets of 4096x4096 (%d MiB), 1 MiB pages"
+                               % (nbytes >> 20), "swaps_per_measurement": n_swap, "parallelism": "single",
+                   "timing": "CUDA events on the swap stream, best of the steps"},
+        "roofline": {"bound": "h2d", "achieved": gbs, "peak": plain_gbs, "unit": "GB/s", "frac": gbs / plain_gbs,
+                     "peak_kind": "measured in this run: plain pinned host-to-device copy of the same bytes",
+                     "traffic": None, "kernel": "copy + swap_in_kernel"},
+        "overlap": {"decode_step_us_alone": dec_ms * 1e3 / n_dec, "decode_step_us_beside_swaps": dec_both * 1e3 / n_dec,
+                    "swap_ms_alone": swap_ms / n_swap, "swap_ms_beside_decode": swap_both / n_swap,
+                    "decode": "q_proj-shaped lora_apply on resident slots, %d steps" % n_dec},
+        "gpu_launches": launches, "clocks": clocks,
+        "cpu_baseline": {"value": None, "unit": "GB/s", "cores": 0, "kind": "none",
+                         "sample": "a host-to-device copy has no CPU oracle; the plain copy is the baseline"},
+    }
     print(json.dumps(line), flush=True)
 
 

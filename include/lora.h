@@ -141,6 +141,39 @@ LORA_API int lora_pool_load(lora_pool *pool, int slot, int target, int rank,
                    const void *A, const void *B, int src_is_device,
                    void *stream);
 
+/*
+ * Swap one adapter in from host memory for all targets at once, without the
+ * host waiting: the adapter's weights move across the host link in one copy
+ * into the caller's device staging area, then one kernel scatters them into
+ * the slot's pages (A rows as given, B transposed, rank padding zeroed), all
+ * in stream order.  The pages' home is the unified page pool ("Multi-LoRA
+ * Serving: Sharing One GPU Across Adapters", section "How S-LoRA Proved the
+ * Model": adapters move between host and GPU memory on demand).
+ *   ranks    host int [n_targets]: the adapter's rank on each target (0 =
+ *            not adapted there), each <= r_max
+ *   src      host memory (pinned, for the copy to run asynchronously) of
+ *            lora_swap_src_bytes(ranks) bytes: for each target t in order with
+ *            ranks[t] > 0, A_t bf16 [rank, d_in] then B_t bf16 [d_out, rank],
+ *            row-major, packed
+ *   staging  device memory, 256-byte aligned, of at least
+ *            lora_swap_staging_bytes(ranks) bytes; it must stay untouched
+ *            until the stream has passed the call
+ * The first load into an empty slot takes its pages from the free list.  The
+ * call must not race with compute calls that read the same slot; compute on
+ * other slots may run concurrently on other streams.  Errors: LORA_ERR_SLOT,
+ * LORA_ERR_INVALID_ARG (rank out of range, src_bytes not the packed size),
+ * LORA_ERR_ALIGNMENT, LORA_ERR_WORKSPACE (staging too small),
+ * LORA_ERR_NO_PAGES, LORA_ERR_CUDA.
+ */
+LORA_API int lora_pool_swap_in(lora_pool *pool, int slot, const int *ranks, const void *src,
+                      size_t src_bytes, void *staging, size_t staging_bytes, void *stream);
+
+/* Bytes of the packed source of lora_pool_swap_in (0 for an invalid rank). */
+LORA_API size_t lora_swap_src_bytes(const lora_pool *pool, const int *ranks);
+
+/* Staging bytes lora_pool_swap_in needs (0 for an invalid rank). */
+LORA_API size_t lora_swap_staging_bytes(const lora_pool *pool, const int *ranks);
+
 /* Release a slot's pages to the free list and mark it empty (its rows then
  * raise LORA_ERR_NOT_LOADED).  Synchronous with respect to the device. */
 LORA_API int lora_pool_unload(lora_pool *pool, int slot);
