@@ -33,7 +33,7 @@ constexpr int kConsumerWarps = 8;    // decode kernel: 8 warps, each copies and 
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumerThreads;
 constexpr int kClusterCtas = 8;      // CTAs that split one work item (portable cluster)
-constexpr int kMaxStages = 4;        // pipeline depth of the decode kernel
+constexpr int kMaxStages = 4;        // barrier slots of the decode ring (it runs n_stages <= this)
 constexpr int kItemSlots = 8;        // items a warp's copies may run ahead of its compute
 constexpr int kFusedMaxT = 256;      // batches up to this size are grouped inside the decode kernel
 constexpr int kMaxMulti = 4;         // targets sharing x in one decode launch

@@ -25,8 +25,10 @@
 //           multiplied by the B^T columns in TMEM; the epilogue adds s * acc
 //           to y (fetched by TMA) in fp32 and stores bf16 for the tile's own
 //           rows, 8 lanes per 128-byte row.
-// Adapter rows are copied into shared memory with 16-byte cp.async through
-// the page table, one lookup per row.  Every wait is bounded.
+// The shrink's A slice arrives by one bulk copy per rank row (through the
+// page table, pieces at page boundaries) into a row-major staging area and is
+// moved into the MMA layout in shared memory; the expand's B^T columns come
+// by 16-byte cp.async, one page lookup per row.  Every wait is bounded.
 #include <cuda.h>
 
 #include <algorithm>

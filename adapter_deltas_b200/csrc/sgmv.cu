@@ -13,17 +13,20 @@
 // attributes to multi-adapter batches is the adapter bytes (section "How does
 // one batch run 30 different adapters at once?").
 //
-// B200 mapping.  A thread-block cluster of kClusterCtas CTAs owns one work
-// item at a time.  CTA c of the cluster handles slice c of d_in for the shrink
-// (split-K) and slice c of d_out for the expand.  Each CTA streams its slices
-// of A / x and B^T / y through a kStages-deep shared-memory ring filled by 1-D
-// bulk async copies (cp.async.bulk, no multicast) that complete on mbarriers;
-// pool rows are located through the page table, piece by piece at page
-// boundaries.  Shrink partial sums are reduced first across lanes by warp
-// shuffles, then across the cluster through distributed shared memory in a
-// fixed CTA order, so every CTA ends with the same fp32 v (deterministic, and
-// independent of the other rows of the batch).  The expand then adds
+// B200 mapping.  A thread-block cluster of kClusterCtas CTAs (4 for batches
+// with many more items than clusters) owns one work unit -- an item on one
+// target -- at a time.  CTA c of the cluster handles slice c of d_in for the
+// shrink (split-K) and slice c of d_out for the expand.  Each CTA streams its
+// slices of A / x and B^T / y through a two-stage shared-memory ring filled
+// by 1-D bulk async copies (cp.async.bulk, no multicast, one per row slice)
+// that complete on mbarriers; pool rows are located through the page table
+// (pieces at page boundaries).  The shrink and the expand run on warp-level
+// bf16 MMA.  Shrink partial sums are reduced over the warps in shared memory,
+// then across the cluster through distributed shared memory (st.async pushes)
+// in a fixed CTA order, so every CTA ends with the same fp32 v (deterministic,
+// and independent of the other rows of the batch).  The expand then adds
 // scale * (B v) to its y slice in fp32 and stores bf16 (round to nearest even).
+// Batches of up to kFusedMaxT rows are grouped by adapter inside the kernel.
 #include <algorithm>
 #include <climits>
 
@@ -271,17 +274,6 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_
   atomicCAS(status, 0, LORA_ERR_TIMEOUT);
   return false;
 }
-// Per-lane 16-byte asynchronous copy global -> shared (L2 only), and an
-// arrive on an mbarrier once all of this thread's prior copies have landed.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src));
-}
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Barrier of the consumer warps only (named barrier 1).
-__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
 
 // Per-item facts a warp needs while it consumes an item.  Every warp keeps
 // its own copy (it resolved the item itself when it began copying it), so no
