@@ -142,28 +142,43 @@ __global__ void __launch_bounds__(kPlanThreads) plan_ids_kernel(const int32_t *_
   }
 }
 
+// One pass over the segments (one per thread, S <= kPlanThreads): offsets,
+// slot and validity are read together; a block scan places segments, decode
+// items and tensor-core tiles; the decode items of the long segments (for
+// targets the tensor cores cannot serve) and the row order are written from
+// shared-memory copies of the segment table.  Larger S take the same steps
+// in chunks of kPlanThreads segments, reading the table back from the plan.
 __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32_t *__restrict__ seg_off,
                                                                       const int32_t *__restrict__ seg_slot,
                                                                       int S, int T, int mma_min, PoolView pool,
                                                                       PlanView plan, int *status) {
   __shared__ Quad s_warp[32];
   __shared__ int s_bad_id, s_bad_empty;
+  __shared__ int s_start[kPlanThreads + 1], s_row[kPlanThreads];
   const int tid = threadIdx.x;
+  const bool one_pass = S <= kPlanThreads;
   if (tid == 0) {
     s_bad_id = 0;
     s_bad_empty = 0;
   }
   griddep_wait();
   griddep_launch_dependents();
-  __syncthreads();
   // Offsets must be non-decreasing and inside [0, T] (then segments are
-  // disjoint); otherwise the whole plan is empty.
+  // disjoint); otherwise the whole plan is empty.  (In one pass the slot and
+  // its loaded flag are read at the same time.)
+  int b0 = 0, e0 = 0, slot0 = -1, loaded0 = 0;
+  bool malformed = false;
   for (int s = tid; s < S; s += kPlanThreads) {
     const int b = seg_off[s], e = seg_off[s + 1];
-    if (b < 0 || e < b || e > T) s_bad_id = 1;
+    if (b < 0 || e < b || e > T) malformed = true;
+    if (one_pass) {
+      b0 = b;
+      e0 = e;
+      slot0 = seg_slot[s];
+      if (slot0 >= 0 && slot0 < pool.n_slots) loaded0 = pool.loaded[slot0];
+    }
   }
-  __syncthreads();
-  if (s_bad_id) {
+  if (__syncthreads_or(malformed)) {
     if (tid == 0) {
       plan.seg_start[0] = 0;
       plan.hdr[kHdrSegs] = 0;
@@ -181,14 +196,23 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
     const int s = base + tid;
     int b = 0, len = 0, slot = -1;
     if (s < S) {
-      b = seg_off[s];
-      const int e = seg_off[s + 1];
-      slot = seg_slot[s];
+      int e, ld;
+      if (one_pass) {
+        b = b0;
+        e = e0;
+        slot = slot0;
+        ld = loaded0;
+      } else {
+        b = seg_off[s];
+        e = seg_off[s + 1];
+        slot = seg_slot[s];
+        ld = (slot >= 0 && slot < pool.n_slots) ? pool.loaded[slot] : 0;
+      }
       if (slot == -1 || e == b) {
         // no adapter, or an empty segment: nothing to do
       } else if (slot < -1 || slot >= pool.n_slots) {
         s_bad_id = 1;
-      } else if (!pool.loaded[slot]) {
+      } else if (!ld) {
         s_bad_empty = 1;
       } else {
         len = e - b;
@@ -205,10 +229,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
       plan.seg_start[seg] = off;
       plan.seg_slot[seg] = slot;
       plan.seg_row[seg] = b;
+      if (one_pass) {
+        s_start[seg] = off;
+        s_row[seg] = b;
+      }
       if (mma) {
         const int j0 = carry.d + ex.d;
-        for (int k = 0; k * kMmaRows < len; ++k)
-          plan.tiles[j0 + k] = make_int4(slot, b + k * kMmaRows, min(kMmaRows, len - k * kMmaRows), seg);
+        for (int k = 0; k * kMmaRows < len; ++k) {
+          const int m = min(kMmaRows, len - k * kMmaRows);
+          plan.tiles[j0 + k] = make_int4(slot, b + k * kMmaRows, m, seg);
+          if (one_pass)  // its decode items, after all the short segments' ones
+            for (int q = 0; q < kMmaRows / kItemRows; ++q)
+              plan.items[tot.c + (j0 + k) * (kMmaRows / kItemRows) + q] =
+                  make_int4(slot, off + k * kMmaRows + q * kItemRows, max(0, min(kItemRows, m - q * kItemRows)), seg);
+        }
       } else {
         const int i0 = carry.c + ex.c;
         for (int k = 0; k * kItemRows < len; ++k)
@@ -217,20 +251,22 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
     }
     carry = quad_add(carry, tot);
   }
-  __syncthreads();
-  // Decode items for the long segments too (after the short ones): targets
-  // the tensor-core path cannot serve take every segment on the decode path.
-  // Each tile of kMmaRows rows becomes kMmaRows / kItemRows items.
   const int n_tiles = carry.d, n_short = carry.c;
-  for (int idx = tid; idx < n_tiles * (kMmaRows / kItemRows); idx += kPlanThreads) {
-    const int j = idx / (kMmaRows / kItemRows), q = idx - j * (kMmaRows / kItemRows);
-    const int4 t = plan.tiles[j];
-    const int first = t.y - plan.seg_row[t.w] + plan.seg_start[t.w] + q * kItemRows;  // perm index
-    const int m = min(kItemRows, t.z - q * kItemRows);
-    plan.items[n_short + idx] = m > 0 ? make_int4(t.x, first, m, t.w) : make_int4(t.x, first, 0, t.w);
+  if (!one_pass) {
+    // Decode items for the long segments too (after the short ones).  Each
+    // tile of kMmaRows rows becomes kMmaRows / kItemRows items.
+    __syncthreads();
+    for (int idx = tid; idx < n_tiles * (kMmaRows / kItemRows); idx += kPlanThreads) {
+      const int j = idx / (kMmaRows / kItemRows), q = idx - j * (kMmaRows / kItemRows);
+      const int4 t = plan.tiles[j];
+      const int first = t.y - plan.seg_row[t.w] + plan.seg_start[t.w] + q * kItemRows;  // perm index
+      const int m = min(kItemRows, t.z - q * kItemRows);
+      plan.items[n_short + idx] = m > 0 ? make_int4(t.x, first, m, t.w) : make_int4(t.x, first, 0, t.w);
+    }
   }
   if (tid == 0) {
     plan.seg_start[carry.b] = carry.a;
+    if (one_pass) s_start[carry.b] = carry.a;
     plan.hdr[kHdrSegs] = carry.b;
     plan.hdr[kHdrActive] = carry.a;
     plan.hdr[kHdrItems] = carry.c;
@@ -241,14 +277,16 @@ __global__ void __launch_bounds__(kPlanThreads) plan_segments_kernel(const int32
   __syncthreads();
   // perm: the rows of segment g are seg_row[g] .. seg_row[g] + length - 1
   const int n_segs = carry.b, n_active = carry.a;
+  const int *starts = one_pass ? s_start : plan.seg_start;
+  const int *rows = one_pass ? s_row : plan.seg_row;
   for (int p = tid; p < n_active; p += kPlanThreads) {
     int lo = 0, hi = n_segs - 1;
     while (lo < hi) {  // last segment whose start is <= p
       const int mid = (lo + hi + 1) >> 1;
-      if (plan.seg_start[mid] <= p) lo = mid;
+      if (starts[mid] <= p) lo = mid;
       else hi = mid - 1;
     }
-    plan.perm[p] = plan.seg_row[lo] + (p - plan.seg_start[lo]);
+    plan.perm[p] = rows[lo] + (p - starts[lo]);
   }
   if (tid == 0) {
     if (s_bad_id) set_status(status, LORA_ERR_BAD_ID);
