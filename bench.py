@@ -86,8 +86,8 @@ def traffic_from_profile(kernel: str, kernel_file: str, workload: str):
     if kv.get("source_sha256") != hashlib.sha256(src).hexdigest():
         return None
     try:
-        return int(kv["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return int(kv["traffic_bytes_per_launch"].split()[0])
+    except (KeyError, ValueError, IndexError):
         return None
 
 
