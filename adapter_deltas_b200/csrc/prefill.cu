@@ -72,6 +72,7 @@ struct __align__(64) PrefillArgs {
   int *status;
   float *vpart;         // [n_ks][T][r_cap] fp32 partial V of each k-slice
   int r_cap;            // 16 or 32
+  int pool_r_max;       // rank rows of a slot's blocks (<= r_cap)
   int kb_per;           // x blocks per k-slice
   int n_ks;             // k-slices
   int n_stages;         // shrink ring stages
@@ -231,7 +232,8 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
   const uint32_t lbo_a = (uint32_t)(a.r_cap / 8) * 128u;  // k-group stride of the A_a slice
   const uint32_t aw_u = smem_u32(S.aw), ring_u = smem_u32(S.ring);
   uint32_t gbase = 0;   // ring uses so far: use g sits in stage g % NS with phase (g / NS) & 1
-  uint32_t ucount = 0;  // units multiplied so far (w_full / a_land / sh_done phases)
+  uint32_t ucount = 0;  // units multiplied so far (w_full / sh_done phases)
+  uint32_t ucopy = 0;   // units whose A slice was copied (a_land phases)
 
   for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
     const int tile = u / a.n_ks, ks = u - tile * a.n_ks;
@@ -256,6 +258,20 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
       __syncwarp();
       gbase += nkb;
       continue;
+    }
+    // The A slice does not wait for the rank: all r_cap rows come (the pool
+    // keeps an adapter's rows past its rank at zero), so the copies leave as
+    // soon as the tile record is known.
+    const int cols = min(nkb * kBoxCols, a.d_in - kb0 * kBoxCols);
+    const uint32_t row_bytes = (uint32_t)cols * 2u, stg_pitch = (uint32_t)a.kb_per * kBoxCols * 2u;
+    const long long row_off0 = a.a_off + (long long)kb0 * kBoxCols * 2;
+    const int rows_cp = min(a.r_cap, a.pool_r_max);
+    if (warp == 0) {
+      if (lane == 0) mbar_arrive_expect_tx(S.a_land, (uint32_t)rows_cp * row_bytes);
+      __syncwarp();
+      if (lane < rows_cp)
+        copy_pool_row(a.pool, slot, row_off0 + (long long)lane * a.d_in * 2, row_bytes, S.stg + lane * stg_pitch,
+                      S.a_land, a.status);
     }
     const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
     const bool use = r > 0 && r <= a.r_cap;
@@ -285,30 +301,28 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
         if (use) mma_commit(S.sh_done);
       }
       __syncwarp();
-    } else if (use) {
+    } else {
       // ------------------------------------------------ epilogue warps
-      // (1) the k-slice of A_a: rows < r by one bulk copy each (pieces where
-      // a row crosses a page) into a row-major staging area, then moved into
-      // the MMA's K-major core-matrix layout, with zero rows up to R and zero
-      // columns beyond d_in
-      const int cols = min(nkb * kBoxCols, a.d_in - kb0 * kBoxCols);
-      const uint32_t row_bytes = (uint32_t)cols * 2u, stg_pitch = (uint32_t)a.kb_per * kBoxCols * 2u;
-      const long long row_off0 = a.a_off + (long long)kb0 * kBoxCols * 2;
-      if (warp == 0) {
-        if (lane == 0) mbar_arrive_expect_tx(S.a_land, (uint32_t)r * row_bytes);
-        __syncwarp();
-        if (lane < r)
-          copy_pool_row(a.pool, slot, row_off0 + (long long)lane * a.d_in * 2, row_bytes, S.stg + lane * stg_pitch,
-                        S.a_land, a.status);
+      // (1) the k-slice of A_a, copied above into a row-major staging area
+      // (one bulk copy per row, pieces where a row crosses a page), moved
+      // into the MMA's K-major core-matrix layout: 8 rank rows x 4 chunks per
+      // warp access, so each 128-byte core matrix is written whole; zero rows
+      // from r up to R and zero columns beyond d_in
+      warp_wait(S.a_land, ucopy & 1u, a.status, alive);
+      if (use) {
+        const int kv_n = nkb * (kBoxCols / 8);
+        const int jl = lane & 7, vo = lane >> 3;
+        for (int jg = 0; jg < R / 8; ++jg) {
+          const int j = jg * 8 + jl;
+          for (int kv = warp * 4 + vo; kv < kv_n; kv += kShEpiWarps * 4) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (j < r && kv * 8 < cols) v = *reinterpret_cast<const uint4 *>(S.stg + j * stg_pitch + kv * 16);
+            *reinterpret_cast<uint4 *>(S.aw + kv * lbo_a + jg * 128 + jl * 16) = v;
+          }
+        }
       }
-      warp_wait(S.a_land, par, a.status, alive);
-      const int kv_n = nkb * (kBoxCols / 8);
-      for (int idx = tid; idx < R * kv_n; idx += kShEpiThreads) {
-        const int j = idx / kv_n, kv = idx - j * kv_n;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (j < r && kv * 8 < cols) v = *reinterpret_cast<const uint4 *>(S.stg + j * stg_pitch + kv * 16);
-        *reinterpret_cast<uint4 *>(S.aw + kv * lbo_a + (j >> 3) * 128 + (j & 7) * 16) = v;
-      }
+    }
+    if (use && warp < kShEpiWarps) {
       fence_async_smem();  // generic-proxy writes -> visible to the MMAs (async proxy)
       tc_fence_before();   // the previous unit's TMEM reads are done
       pf_arrive(S.w_full);
@@ -330,8 +344,12 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
         }
       }
     }
+    // the epilogue warps stay in step (an absent adapter's unit has no
+    // other barrier that would hold them together)
+    if (warp < kShEpiWarps) asm volatile("bar.sync 1, %0;" ::"n"(kShEpiThreads) : "memory");
     gbase += nkb;
     if (use) ++ucount;
+    ++ucopy;
   }
 
   tc_fence_before();
@@ -684,6 +702,7 @@ int launch_prefill(lora_pool *pool, int target, const void *x, int ldx, void *y,
   a.status = pool->d_status;
   a.vpart = reinterpret_cast<float *>(static_cast<uint8_t *>(const_cast<void *>(ws)) + plan_bytes);
   a.r_cap = geo.r_cap;
+  a.pool_r_max = pool->r_max;
   a.kb_per = geo.kb_per;
   a.n_ks = geo.n_ks;
   a.n_stages = geo.n_stages;
