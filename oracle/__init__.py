@@ -18,6 +18,10 @@ Functions and the passages they follow (pages on multi-LoRA serving):
   and "Batching across adapters" (per-row correction), worked example
   (adapter=None leaves the base output).
 * ``lora_expand``  -- the second factor of the same formula, given v = A x.
+* ``linear`` / ``lora_linear`` -- the shared base term xW of the same
+  formula (W stored d_out x d_in as in the column form W.x of "Serving Many
+  LoRA Adapters From One Base Model", section "How it works"), and the whole
+  layer output xW + (x A_i) B_i alpha/r.
 * ``group_rows``   -- "Multi-LoRA Serving: Why 100 Adapters Fit on One GPU",
   section "How does one batch run 30 different adapters at once?" (index
   vector, segmented gather).
@@ -76,6 +80,8 @@ def _load():
     lib.oracle_pool_locate.argtypes = [I, ctypes.c_longlong, P, I, ctypes.c_longlong]
     lib.oracle_slot_layout.restype = ctypes.c_longlong
     lib.oracle_slot_layout.argtypes = [I, P, P, I, P, P]
+    lib.oracle_linear.restype = None
+    lib.oracle_linear.argtypes = [I, I, I, P, P, P, I]
     lib.oracle_lora_params.restype = ctypes.c_longlong
     lib.oracle_lora_params.argtypes = [ctypes.c_longlong] * 4
     _lib = lib
@@ -177,6 +183,27 @@ def lora_expand(v, y_in, ids, n_slots: int, B_by_slot: Dict[int, np.ndarray],
                                  _ptr(alpha64), _ptr(out))
     del keep
     return out, bad
+
+
+def linear(x, W, threads: int = 1) -> np.ndarray:
+    """out[t] = W x[t] (the base term xW with W stored [d_out, d_in]), fp64."""
+    lib = _load()
+    x64 = _as_f64(x)
+    W64 = _as_f64(W)
+    T, d_in = x64.shape
+    d_out = W64.shape[0]
+    assert W64.shape[1] == d_in, "W is d_out x d_in"
+    out = np.empty((T, d_out), dtype=np.float64)
+    lib.oracle_linear(T, d_in, d_out, _ptr(x64), _ptr(W64), _ptr(out), threads)
+    return out
+
+
+def lora_linear(x, W, ids, n_slots: int, adapters: Adapters,
+                alpha: Sequence[float], threads: int = 1):
+    """The whole layer: y[t] = W x[t] + (alpha_a / r_a) B_a (A_a x[t]), a = ids[t]
+    (rows without a valid adapter get W x[t] alone).  Returns (y fp64, number
+    of rows with an invalid id)."""
+    return lora_apply(x, linear(x, W, threads), ids, n_slots, adapters, alpha, threads)
 
 
 def group_rows(ids, n_slots: int, valid: Optional[np.ndarray] = None):

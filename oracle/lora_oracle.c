@@ -160,6 +160,61 @@ int oracle_lora_apply(int T, int d_in, int d_out,
     return bad;
 }
 
+/* ---------------------------------------------------------------------- */
+/* The shared base term, fp64.                                             */
+/* ---------------------------------------------------------------------- */
+
+typedef struct {
+    int t_begin, t_end, d_in, d_out;
+    const double *x;   /* [T][d_in] */
+    const double *W;   /* [d_out][d_in] */
+    double *out;       /* [T][d_out] */
+} linear_job;
+
+static void *linear_rows(void *arg)
+{
+    linear_job *j = (linear_job *)arg;
+    for (int t = j->t_begin; t < j->t_end; ++t) {
+        const double *xt = j->x + (size_t)t * j->d_in;
+        for (int n = 0; n < j->d_out; ++n) {
+            const double *wn = j->W + (size_t)n * j->d_in;
+            double acc = 0.0;
+            for (int k = 0; k < j->d_in; ++k) acc += xt[k] * wn[k];
+            j->out[(size_t)t * j->d_out + n] = acc;
+        }
+    }
+    return NULL;
+}
+
+/*
+ * out[t][n] = sum_k x[t][k] * W[n][k]: the base term xW that every row shares
+ * ("Multi-LoRA Serving: Why 100 Adapters Fit on One GPU", section "Why can't
+ * you just merge LoRA weights into the base model?").  W is stored as the
+ * d_out x d_in matrix of the column form W.x ("Serving Many LoRA Adapters
+ * From One Base Model", section "How it works"), so the row form's xW is the
+ * product of x with the transpose of this W.  Rows are split over n_threads
+ * threads; each output is one k-ascending dot product whatever the count.
+ */
+void oracle_linear(int T, int d_in, int d_out, const double *x,
+                   const double *W, double *out, int n_threads)
+{
+    if (T <= 0) return;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > T) n_threads = T;
+    linear_job *jobs = (linear_job *)calloc((size_t)n_threads, sizeof(linear_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)n_threads, sizeof(pthread_t));
+    for (int i = 0; i < n_threads; ++i) {
+        linear_job *j = &jobs[i];
+        j->t_begin = (int)((long long)T * i / n_threads);
+        j->t_end = (int)((long long)T * (i + 1) / n_threads);
+        j->d_in = d_in; j->d_out = d_out; j->x = x; j->W = W; j->out = out;
+    }
+    for (int i = 1; i < n_threads; ++i) pthread_create(&th[i], NULL, linear_rows, &jobs[i]);
+    linear_rows(&jobs[0]);
+    for (int i = 1; i < n_threads; ++i) pthread_join(th[i], NULL);
+    free(jobs); free(th);
+}
+
 /*
  * Expand step alone: y_out[t] = y_in[t] + (alpha_a / r_a) * B_a v[t], with the
  * caller's v[t] (first r_a entries of row t of a [T][ldv] array).  Same row

@@ -176,6 +176,54 @@ def test_integer_brute_force_exact():
             assert Fraction(y[t, n]) == ref, (t, n)
 
 
+# ---------------------------------------------------------------- base term
+
+
+def test_linear_is_a_library_matmul():
+    # the base term xW against numpy's matmul (W stored d_out x d_in)
+    g = np.random.default_rng(11)
+    x = g.standard_normal((7, 33))
+    W = g.standard_normal((19, 33))
+    ref = x @ W.T
+    got = oracle.linear(x, W, threads=3)
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=1e-13 * np.abs(ref).max())
+    # a transposed operand would give another shape or other values
+    assert got.shape == (7, 19)
+
+
+def test_linear_integer_brute_force_exact():
+    g = np.random.default_rng(12)
+    x = g.integers(-4, 5, size=(3, 6)).astype(np.float64)
+    W = g.integers(-3, 4, size=(5, 6)).astype(np.float64)
+    got = oracle.linear(x, W)
+    for t in range(3):
+        for n in range(5):
+            assert got[t, n] == sum(int(x[t, k]) * int(W[n, k]) for k in range(6))
+
+
+def test_lora_linear_equals_merged_weight_per_row():
+    # the whole layer: row t equals x[t] (W + (alpha_a/r_a) B_a A_a)^T, the
+    # merged form, and the plain base for rows without an adapter
+    x, W, _, adapters, ids, alpha = _rand_case(13, 17, 24, 40, [3, 5, 1], [6.0, 2.5, 7.0])
+    y, bad = oracle.lora_linear(x, W, ids, 3, adapters, alpha, threads=2)
+    assert bad == 0
+    for t in range(x.shape[0]):
+        a = ids[t]
+        Wm = W
+        if a >= 0:
+            A, B = adapters[a]
+            Wm = W + (alpha[a] / A.shape[0]) * (B @ A)
+        ref = x[t] @ Wm.T
+        np.testing.assert_allclose(y[t], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_lora_linear_without_adapters_is_the_base():
+    x, W, _, adapters, ids, alpha = _rand_case(14, 9, 16, 8, [2], [4.0])
+    none = np.full(9, -1, np.int32)
+    y, bad = oracle.lora_linear(x, W, none, 1, adapters, alpha)
+    assert bad == 0 and np.array_equal(y, oracle.linear(x, W))
+
+
 def test_unit_vector_expand_is_a_column_of_B():
     # v = e_j  ->  delta = (alpha/r) * column j of B
     g = np.random.default_rng(7)
