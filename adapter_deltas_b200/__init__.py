@@ -78,6 +78,7 @@ _sig("lora_pool_page_table", _P, [_P])
 _sig("lora_pool_get_info", _I, [_P, ctypes.POINTER(lora_pool_info)])
 _sig("lora_pool_target_offsets", _I, [_P, _I, ctypes.POINTER(_Z), ctypes.POINTER(_Z)])
 _sig("lora_workspace_bytes", _Z, [_P, _I, _I])
+_sig("lora_linear_workspace_bytes", _Z, [_P, _I, _I])
 _sig("lora_plan_layout_get", _I, [_P, _I, ctypes.POINTER(lora_plan_layout)])
 _sig("lora_plan_ids", _I, [_P, _P, _I, _P, _Z, _P])
 _sig("lora_plan_segments", _I, [_P, _P, _P, _I, _I, _P, _Z, _P])
@@ -86,6 +87,7 @@ _sig("lora_apply_plan", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_apply", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_segments", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_apply_multi", _I, [_P, _I, _P, _P, _I, _P, _I, _P, _P, _P, _I, _P, _Z, _P])
+_sig("lora_linear", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_shrink", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_noalloc", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
@@ -284,6 +286,16 @@ def lora_apply_segments(pool: PoolHandle, target: int, x, y, seg_offsets, seg_sl
     _check(_lib.lora_apply_segments(pool, target, _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(seg_offsets),
                                     _ptr(seg_slot), seg_slot.shape[0], _ptr(scales), y.shape[0], _ptr(ws),
                                     ws.numel(), _stream(stream)), "lora_apply_segments")
+
+
+def lora_linear_workspace_bytes(pool: PoolHandle, target: int, max_tokens: int) -> int:
+    return int(_lib.lora_linear_workspace_bytes(pool, target, max_tokens))
+
+
+def lora_linear(pool: PoolHandle, target: int, x, W, y, ids, scales, ws, stream=None) -> None:
+    """y = x W^T + each row's delta, written once (W: [d_out, d_in] row-major)."""
+    _check(_lib.lora_linear(pool, target, _ptr(x), _ld(x), _ptr(W), _ld(W), _ptr(y), _ld(y), _ptr(ids),
+                            _ptr(scales), y.shape[0], _ptr(ws), ws.numel(), _stream(stream)), "lora_linear")
 
 
 def lora_shrink(pool: PoolHandle, target: int, x, ids, v, ws, stream=None) -> None:

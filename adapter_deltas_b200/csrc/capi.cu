@@ -219,4 +219,40 @@ int lora_expand(lora_pool *p, int target, const float *v, int ldv, void *y, int 
                        static_cast<cudaStream_t>(stream));
 }
 
+size_t lora_linear_workspace_bytes(const lora_pool *p, int target, int max_tokens) {
+  if (!p || target < 0 || target >= p->n_targets || max_tokens < 0 || max_tokens > kMaxTokens) return 0;
+  return align256(plan_layout(max_tokens).total) + align256(size_t(max_tokens) * p->r_max * 4);
+}
+
+int lora_linear(lora_pool *p, int target, const void *x, int ldx, const void *W, int ldw, void *y, int ldy,
+                const int32_t *ids, const float *scales, int T, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_call(p, target, T, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  const int d_in = p->targets[target].d_in, d_out = p->targets[target].d_out;
+  if ((rc = check_rows(x, ldx, d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, d_out)) != LORA_OK) return rc;
+  if ((rc = check_rows(W, ldw, d_in)) != LORA_OK) return rc;
+  if (!ids || !scales) return LORA_ERR_INVALID_ARG;
+  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  {
+    const char *wa = static_cast<const char *>(W), *ya = static_cast<const char *>(y);
+    if (wa < ya + size_t(T) * ldy * 2 && ya < wa + size_t(d_out) * ldw * 2) return LORA_ERR_INVALID_ARG;
+  }
+  const size_t voff = align256(plan_layout(T).total);
+  if (ws_bytes < voff + size_t(T) * p->r_max * 4) return LORA_ERR_WORKSPACE;
+  float *v = reinterpret_cast<float *>(static_cast<char *>(ws) + voff);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T <= kFusedMaxT) {
+    DeviceGuard g(p->device);
+    rc = launch_decode_ids(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, p->r_max, ids, T, st);
+  } else {
+    if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
+    DeviceGuard g(p->device);
+    rc = launch_decode(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, p->r_max, T, ws, st);
+  }
+  if (rc != LORA_OK) return rc;
+  DeviceGuard g(p->device);
+  return launch_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, v, p->r_max, T, st);
+}
+
 }  // extern "C"

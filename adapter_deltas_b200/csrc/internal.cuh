@@ -338,5 +338,9 @@ size_t prefill_scratch_bytes(const lora_pool *pool, int target, int T);
 int launch_prefill(lora_pool *pool, int target, const void *x, int ldx, void *y, int ldy, const float *scales,
                    int T, const void *ws, size_t ws_bytes, cudaStream_t st);
 int decode_setup(lora_pool *pool);
+// Base projection fused with the delta (linear.cu): y = W x + s_a B_a v, v the
+// shrink's fp32 output [T, ldv].
+int launch_linear(lora_pool *pool, int target, const void *x, int ldx, const void *W, int ldw, void *y, int ldy,
+                  const int32_t *ids, const float *scales, const float *v, int ldv, int T, cudaStream_t st);
 
 }  // namespace lora

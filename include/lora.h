@@ -324,6 +324,41 @@ LORA_API int lora_apply_multi(lora_pool *pool, int n_targets, const int *targets
                      const int32_t *ids, const float *scales, int T, void *ws,
                      size_t ws_bytes, void *stream);
 
+/* ------------------------------------------ the layer with its delta fused */
+
+/*
+ * The whole projection layer with each row's adapter, y written once:
+ *     y[t, n] = bf16( sum_k W[n, k] x[t, k] + scales[a] * (B_a (A_a x[t]))[n] ),
+ * a = ids[t]; rows with no adapter (id -1, a bad id, an empty slot, rank 0 on
+ * this target) get the base term alone.  This is y = xW + (x A_i) B_i alpha/r
+ * of "Multi-LoRA Serving: Why 100 Adapters Fit on One GPU", section "Why
+ * can't you just merge LoRA weights into the base model?", with W stored as
+ * the d_out x d_in matrix of the column form W.x ("Serving Many LoRA Adapters
+ * From One Base Model", section "How it works").  The delta is accumulated in
+ * fp32 together with the base product and rounded once; unlike lora_apply, y
+ * is only written.
+ *   x, ldx     device bf16 [T, ldx], ldx >= d_in, multiple of 8
+ *   W, ldw     device bf16 [d_out, ldw] row-major (one row per output
+ *              feature), ldw >= d_in, multiple of 8; caller-owned, read only
+ *   y, ldy     device bf16 [T, ldy], ldy >= d_out, multiple of 8; written;
+ *              may overlap neither x nor W
+ *   ids, scales, T, stream  as for lora_apply
+ *   ws, ws_bytes  device workspace of at least lora_linear_workspace_bytes
+ *              (the plan, then v = A_a x[t] in fp32)
+ * Two launches for up to 256 rows (the shrink, then one tensor-core kernel
+ * that streams W and adds the delta inside its accumulator), three beyond
+ * (plan, shrink, that kernel).  Errors: as for lora_apply, and
+ * LORA_ERR_INVALID_ARG for overlapping x / W / y.  The sticky device status
+ * reports bad ids and empty slots as for lora_apply.
+ */
+LORA_API int lora_linear(lora_pool *pool, int target, const void *x, int ldx, const void *W,
+                int ldw, void *y, int ldy, const int32_t *ids, const float *scales,
+                int T, void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace of lora_linear for up to max_tokens rows on `target` (0 for bad
+ * arguments). */
+LORA_API size_t lora_linear_workspace_bytes(const lora_pool *pool, int target, int max_tokens);
+
 /* lora_plan_segments followed by lora_apply_plan. */
 LORA_API int lora_apply_segments(lora_pool *pool, int target, const void *x, int ldx,
                         void *y, int ldy, const int32_t *seg_offsets,

@@ -160,6 +160,19 @@ class Workload:
                 self._cache[key] = normal_bf16(g, (self.T, d_in), 1.0)
         return self._cache[key]
 
+    def W(self, target: int) -> np.ndarray:
+        """Base weight of the target, bf16 bits [d_out, d_in] (one row per
+        output feature): N(0, 1/d_in), or integers in [-2, 2]."""
+        key = ("W", target)
+        if key not in self._cache:
+            d_in, d_out = self.targets[target]
+            g = _rng(self.seed, _T_W, target)
+            if self.value_mode == "integer":
+                self._cache[key] = f32_to_bf16_bits(g.integers(-2, 3, size=(d_out, d_in)).astype(np.float32))
+            else:
+                self._cache[key] = normal_bf16(g, (d_out, d_in), 1.0 / np.sqrt(d_in))
+        return self._cache[key]
+
     def y_in(self, target: int) -> np.ndarray:
         key = ("y", target)
         if key not in self._cache:
@@ -170,9 +183,8 @@ class Workload:
             elif self.y_mode == "normal":
                 y = normal_bf16(_rng(self.seed, _T_Y, target), (self.T, d_out), 1.0)
             else:
-                W = normal_bf16(_rng(self.seed, _T_W, target), (d_out, d_in), 1.0 / np.sqrt(d_in))
                 xf = bf16_bits_to_f32(self.x(target)).astype(np.float64)
-                Wf = bf16_bits_to_f32(W).astype(np.float64)
+                Wf = bf16_bits_to_f32(self.W(target)).astype(np.float64)
                 y = f32_to_bf16_bits((xf @ Wf.T).astype(np.float32))
             self._cache[key] = y
         return self._cache[key]
