@@ -88,6 +88,7 @@ _sig("lora_apply", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_segments", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_apply_multi", _I, [_P, _I, _P, _P, _I, _P, _I, _P, _P, _P, _I, _P, _Z, _P])
 _sig("lora_linear", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
+_sig("lora_linear_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
 _sig("lora_shrink", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_noalloc", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
@@ -296,6 +297,13 @@ def lora_linear(pool: PoolHandle, target: int, x, W, y, ids, scales, ws, stream=
     """y = x W^T + each row's delta, written once (W: [d_out, d_in] row-major)."""
     _check(_lib.lora_linear(pool, target, _ptr(x), _ld(x), _ptr(W), _ld(W), _ptr(y), _ld(y), _ptr(ids),
                             _ptr(scales), y.shape[0], _ptr(ws), ws.numel(), _stream(stream)), "lora_linear")
+
+
+def lora_linear_expand(pool: PoolHandle, target: int, x, W, v, y, ids, scales, stream=None) -> None:
+    """y = x W^T + each row's s_a B_a v[t] (v from lora_shrink), written once."""
+    _check(_lib.lora_linear_expand(pool, target, _ptr(x), _ld(x), _ptr(W), _ld(W), _ptr(v), _ld(v), _ptr(y),
+                                   _ld(y), _ptr(ids), _ptr(scales), y.shape[0], _stream(stream)),
+           "lora_linear_expand")
 
 
 def lora_shrink(pool: PoolHandle, target: int, x, ids, v, ws, stream=None) -> None:

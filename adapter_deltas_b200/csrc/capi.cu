@@ -34,6 +34,22 @@ bool overlap(const void *x, int ldx, const void *y, int ldy, int T) {
   return xa < yb && ya < xb;
 }
 
+// Operands of the fused layer: x [T, d_in], W [d_out, d_in], y [T, d_out];
+// y overlaps neither x nor W.
+int check_linear(const lora_pool *p, int target, const void *x, int ldx, const void *W, int ldw, const void *y,
+                 int ldy, const int32_t *ids, const float *scales, int T) {
+  const int d_in = p->targets[target].d_in, d_out = p->targets[target].d_out;
+  int rc;
+  if ((rc = check_rows(x, ldx, d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, d_out)) != LORA_OK) return rc;
+  if ((rc = check_rows(W, ldw, d_in)) != LORA_OK) return rc;
+  if (!ids || !scales) return LORA_ERR_INVALID_ARG;
+  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  const char *wa = static_cast<const char *>(W), *ya = static_cast<const char *>(y);
+  if (wa < ya + size_t(T) * ldy * 2 && ya < wa + size_t(d_out) * ldw * 2) return LORA_ERR_INVALID_ARG;
+  return LORA_OK;
+}
+
 enum { kPlanUnknown = 0, kPlanIds = 1, kPlanSegments = 2 };
 
 void set_plan_kind(lora_pool *p, const void *ws, int kind) {
@@ -228,31 +244,26 @@ int lora_linear(lora_pool *p, int target, const void *x, int ldx, const void *W,
                 const int32_t *ids, const float *scales, int T, void *ws, size_t ws_bytes, void *stream) {
   int rc = check_call(p, target, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
-  const int d_in = p->targets[target].d_in, d_out = p->targets[target].d_out;
-  if ((rc = check_rows(x, ldx, d_in)) != LORA_OK) return rc;
-  if ((rc = check_rows(y, ldy, d_out)) != LORA_OK) return rc;
-  if ((rc = check_rows(W, ldw, d_in)) != LORA_OK) return rc;
-  if (!ids || !scales) return LORA_ERR_INVALID_ARG;
-  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
-  {
-    const char *wa = static_cast<const char *>(W), *ya = static_cast<const char *>(y);
-    if (wa < ya + size_t(T) * ldy * 2 && ya < wa + size_t(d_out) * ldw * 2) return LORA_ERR_INVALID_ARG;
-  }
+  if ((rc = check_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, T)) != LORA_OK) return rc;
   const size_t voff = align256(plan_layout(T).total);
   if (ws_bytes < voff + size_t(T) * p->r_max * 4) return LORA_ERR_WORKSPACE;
   float *v = reinterpret_cast<float *>(static_cast<char *>(ws) + voff);
+  if ((rc = lora_shrink(p, target, x, ldx, ids, T, v, p->r_max, ws, ws_bytes, stream)) != LORA_OK) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (T <= kFusedMaxT) {
-    DeviceGuard g(p->device);
-    rc = launch_decode_ids(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, p->r_max, ids, T, st);
-  } else {
-    if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
-    DeviceGuard g(p->device);
-    rc = launch_decode(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, p->r_max, T, ws, st);
-  }
-  if (rc != LORA_OK) return rc;
   DeviceGuard g(p->device);
   return launch_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, v, p->r_max, T, st);
+}
+
+int lora_linear_expand(lora_pool *p, int target, const void *x, int ldx, const void *W, int ldw, const float *v,
+                       int ldv, void *y, int ldy, const int32_t *ids, const float *scales, int T, void *stream) {
+  if (!p || target < 0 || target >= p->n_targets || T < 0 || T > kMaxTokens) return LORA_ERR_INVALID_ARG;
+  if (T == 0) return LORA_OK;
+  int rc = check_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, T);
+  if (rc != LORA_OK) return rc;
+  if (!v || ldv < p->r_max) return LORA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(v) & 3u) return LORA_ERR_ALIGNMENT;
+  DeviceGuard g(p->device);
+  return launch_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, v, ldv, T, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

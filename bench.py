@@ -1,7 +1,7 @@
 """Benchmark of the multi-LoRA delta path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload q_proj|tiny|prefill|mlp|paged|qkv|swapin]
+                    [--workload q_proj|tiny|prefill|mlp|paged|qkv|swapin|linear]
 
 Default workload (the metric's configuration): Llama-2-7B q_proj-shaped decode,
 d_in = d_out = 4096, rank 16 for all, 32 resident adapters in a contiguous
@@ -43,7 +43,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "LoRA-delta tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
-WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5, "qkv": 2, "swapin": 5}
+WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5, "qkv": 2, "swapin": 5, "linear": 2}
+LINEAR_WORKLOAD = "q_proj layer with its delta fused: y = x W^T + delta, d4096 r16 32 adapters 64 tokens"
 L2_BYTES = 126 * 2 ** 20
 FUSED_MAX_T = 256   # batches up to this size are grouped inside the decode kernel (one launch)
 
@@ -142,11 +143,17 @@ class ClockSampler:
 # ---------------------------------------------------------------- CPU arms
 
 
-def oracle_inputs(w, target: int):
+def oracle_inputs(w, target: int, layer: bool = False):
     """The oracle's inputs for one batch of one target (drawn once, outside
-    any timed region)."""
+    any timed region); layer: the whole projection (base weight W instead of
+    a given y)."""
     slots = [int(s) for s in np.unique(w.ids[w.ids >= 0])]
-    return dict(x=w.x(target), y=w.y_in(target), adapters={s: w.adapter(s, target) for s in slots})
+    inp = dict(x=w.x(target), adapters={s: w.adapter(s, target) for s in slots})
+    if layer:
+        inp["W"] = w.W(target)
+    else:
+        inp["y"] = w.y_in(target)
+    return inp
 
 
 def time_oracle(w, inp, min_seconds: float, threads: int, max_calls: int = 1 << 30):
@@ -155,10 +162,13 @@ def time_oracle(w, inp, min_seconds: float, threads: int, max_calls: int = 1 << 
     import oracle
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.lora_apply(inp["x"], inp["y"], w.ids, w.n_slots, inp["adapters"], w.alpha, threads=threads)
+        if "W" in inp:
+            oracle.lora_linear(inp["x"], inp["W"], w.ids, w.n_slots, inp["adapters"], w.alpha, threads=threads)
+        else:
+            oracle.lora_apply(inp["x"], inp["y"], w.ids, w.n_slots, inp["adapters"], w.alpha, threads=threads)
         n += 1
         el = time.perf_counter() - t0
-        if el >= min_seconds or n >= max_calls:
+        if (min_seconds > 0 and el >= min_seconds) or n >= max_calls:
             break
     return n, el
 
@@ -181,31 +191,35 @@ def run_reference(args, rank: int, world: int):
     w = synth.config(WORKLOADS[args.workload])
     n_t = len(w.targets) if args.workload == "paged" else 3 if args.workload == "qkv" else 1
     threads = min(cpu_threads(), w.T)
-    inp = oracle_inputs(w, 0)
+    inp = oracle_inputs(w, 0, layer=args.workload == "linear")
     time_oracle(w, inp, 0.0, threads, max_calls=args.warmup)
     n, el = time_oracle(w, inp, 0.0, threads, max_calls=args.steps)
     per_call = el / n
     value = w.T / (per_call * n_t)
     sample = "%d whole batches of %d tokens on target 0" % (n, w.T)
+    if args.workload == "linear":
+        sample += ", whole layer (x W^T + delta)"
     if n_t > 1:
         sample += " (1 of the %d same-shape deltas of a step; value scaled by %d)" % (n_t, n_t)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * per_call * n_t,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w.T, "seq_len": 1, "parallelism": "oracle on host cores"},
+        "config": {"workload": LINEAR_WORKLOAD if args.workload == "linear" else w.name, "global_batch": w.T,
+                   "seq_len": 1, "parallelism": "oracle on host cores"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w, n_targets: int, seconds: float):
+def cpu_baseline(w, n_targets: int, seconds: float, layer: bool = False):
     """The oracle on a bounded sample of the workload (rank 0, N = 1)."""
     threads = min(cpu_threads(), w.T)
-    inp = oracle_inputs(w, 0)
+    inp = oracle_inputs(w, 0, layer)
     n, el = time_oracle(w, inp, seconds, threads)
-    sample = "%d whole batches of %d tokens on target 0 (%.1f s)" % (n, w.T, el)
+    sample = "%d whole batches of %d tokens on target 0%s (%.1f s)" % (
+        n, w.T, ", whole layer (x W^T + delta)" if layer else "", el)
     if n_targets > 1:
         sample += ", value scaled by the %d same-shape deltas of a step" % n_targets
     return {"value": n * w.T / el / n_targets, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -239,6 +253,8 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         return run_qkv(args, rank, world, dev, w, scales, bf16)
     if args.workload == "swapin":
         return run_swapin(args, rank, world, dev, bf16)
+    if args.workload == "linear":
+        return run_linear(args, rank, world, dev, w, scales, bf16)
 
     # one buffer set: pool (all slots loaded), x, y, ids, workspace
     pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
@@ -647,6 +663,162 @@ def run_qkv(args, rank, world, dev, w2, scales, bf16):
     }
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(w, n_t, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def run_linear(args, rank, world, dev, w, scales, bf16):
+    """The q_proj decode batch as a whole projection layer: y = x W^T + each
+    row's delta, W a 4096 x 4096 bf16 base weight.  A step is one
+    lora_linear call (the shrink launch, then the tensor-core layer kernel
+    that streams W and adds the delta inside its accumulator; y written
+    once).  Timed in the same run for context: the base product alone
+    (torch.matmul, cuBLAS) and the unfused layer (that product, then
+    lora_apply adding the delta to y in place)."""
+    import torch
+
+    import adapter_deltas_b200 as L
+    target = 0
+    d_in, d_out = w.targets[target]
+    T = w.T
+    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
+    set_bytes = pool_bytes + d_out * d_in * 2 + T * (d_in + d_out) * 2
+    n_sets = max(2, min(32, -(-4 * L2_BYTES // set_bytes)))
+    adapters = {}
+    for s_ in range(w.n_slots):
+        if w.rank[s_] > 0:
+            A, B = w.adapter(s_, target)
+            adapters[s_] = (bf16(A), bf16(B))
+    W0, x0, ids0 = bf16(w.W(target)), bf16(w.x(target)), torch.from_numpy(w.ids).to(dev)
+    sets = []
+    for k in range(n_sets):
+        mem = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
+        pool = L.lora_pool_create(dev.index, w.targets, w.r_max, w.n_slots, w.page_bytes, mem, w.scatter_seed)
+        for s_, (A, B) in adapters.items():
+            L.lora_pool_load(pool, s_, target, int(w.rank[s_]), A, B)
+        sets.append(dict(pool=pool, mem=mem, W=W0.clone(), x=x0.clone(), ids=ids0.clone(),
+                         y=torch.empty(T, d_out, dtype=torch.bfloat16, device=dev),
+                         v=torch.zeros(T, w.r_max, dtype=torch.float32, device=dev),
+                         ws=torch.zeros(L.lora_linear_workspace_bytes(pool, target, T), dtype=torch.uint8,
+                                        device=dev),
+                         ws_apply=torch.zeros(L.lora_workspace_bytes(pool, target, T), dtype=torch.uint8,
+                                              device=dev)))
+    for s_ in sets:   # v of each set, for the layer kernel timed alone
+        L.lora_shrink(s_["pool"], target, s_["x"], s_["ids"], s_["v"], s_["ws_apply"])
+    torch.cuda.synchronize()
+
+    def step(k):
+        s_ = sets[k % n_sets]
+        L.lora_linear(s_["pool"], target, s_["x"], s_["W"], s_["y"], s_["ids"], scales, s_["ws"])
+
+    def layer_kernel(k):
+        s_ = sets[k % n_sets]
+        L.lora_linear_expand(s_["pool"], target, s_["x"], s_["W"], s_["v"], s_["y"], s_["ids"], scales)
+
+    def base_only(k):
+        s_ = sets[k % n_sets]
+        torch.matmul(s_["x"], s_["W"].t(), out=s_["y"])
+
+    def unfused(k):
+        s_ = sets[k % n_sets]
+        torch.matmul(s_["x"], s_["W"].t(), out=s_["y"])
+        L.lora_apply(s_["pool"], target, s_["x"], s_["y"], s_["ids"], scales, s_["ws_apply"])
+
+    def timed(fn, n):
+        g_w, _ = capture_graph(dev, fn, range(args.warmup))
+        g, launches = capture_graph(dev, fn, range(n))
+        g_w.replay()
+        torch.cuda.synchronize()
+        sync_ranks(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        g.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        sync_ranks(world)
+        del g, g_w
+        return reduce_max(ev0.elapsed_time(ev1) / n, world, dev), launches
+
+    # cuBLAS creates its handle on first use, which a graph capture refuses
+    side = torch.cuda.Stream(dev)
+    with torch.cuda.stream(side):
+        unfused(0)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        ms, launches = timed(step, args.steps)
+    clocks = sampler.stop()
+    reps = max(args.steps, 3 * n_sets)
+    kernel_ms, _ = timed(layer_kernel, reps)
+    base_ms, _ = timed(base_only, reps)
+    unfused_ms, _ = timed(unfused, args.steps)
+
+    # end to end through the C ABI: x and ids in from one packed pinned
+    # buffer, y out, every step (W and the adapters stay resident)
+    parts = [ids0.cpu().view(torch.uint8), x0.cpu().view(torch.uint8).reshape(-1)]
+    offs, total = [], 0
+    for t_ in parts:
+        offs.append(total)
+        total += -(-t_.numel() // 256) * 256
+    packed_h = torch.zeros(total, dtype=torch.uint8).pin_memory()
+    for o, t_ in zip(offs, parts):
+        packed_h[o:o + t_.numel()] = t_
+    yout = torch.empty(T, d_out, dtype=torch.bfloat16).pin_memory()
+    packed_d = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(n_sets)]
+
+    def e2e_step(k):
+        s_ = sets[k % n_sets]
+        buf = packed_d[k % n_sets]
+        buf.copy_(packed_h, non_blocking=True)
+        ids = buf[offs[0]:offs[0] + T * 4].view(torch.int32)
+        x = buf[offs[1]:offs[1] + T * d_in * 2].view(torch.bfloat16).view(T, d_in)
+        L.lora_linear(s_["pool"], target, x, s_["W"], s_["y"], ids, scales, s_["ws"])
+        yout.copy_(s_["y"], non_blocking=True)
+
+    e2e_ms, _ = timed(e2e_step, args.steps)
+    for s_ in sets:
+        L.lora_pool_destroy(s_["pool"])
+    if rank != 0:
+        return
+    peak, peak_kind = load_peaks()
+    act = w.ids[w.ids >= 0]
+    distinct = np.unique(act)
+    # the layer kernel: W, x, y written once, B of each distinct adapter and
+    # v of the adapted rows; the whole step adds each adapter's A, x again
+    # for the shrink and v written
+    w_bytes = d_out * d_in * 2
+    b_bytes = int(sum(int(w.rank[a]) * d_out * 2 for a in distinct))
+    a_bytes = int(sum(int(w.rank[a]) * d_in * 2 for a in distinct))
+    v_bytes = int(sum(int(w.rank[a]) * 4 for a in act))
+    alg_kernel = w_bytes + T * d_in * 2 + T * d_out * 2 + b_bytes + v_bytes
+    alg_step = alg_kernel + a_bytes + act.size * d_in * 2 + v_bytes
+    achieved = alg_kernel / (kernel_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": job_value(T, world, ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": LINEAR_WORKLOAD, "global_batch": T * world, "seq_len": 1,
+                   "parallelism": "replicas%d" % world if world > 1 else "single",
+                   "l2": "%d rotating buffer sets (own W, pool, x, y), %.0f MB > 4x L2" % (
+                       n_sets, n_sets * set_bytes / 1e6),
+                   "timing": "CUDA graph of the K steps, CUDA events around its replay"},
+        "hbm_gbs_step": alg_step / (ms * 1e-3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": traffic_from_profile("linear_kernel", "linear.cu", "linear"),
+                     "traffic_note": "DRAM bytes of one launch from the ncu summary in profiles/, while its "
+                                     "source hash matches",
+                     "kernel": "linear_kernel (tcgen05: W streamed by TMA, delta in the accumulator), "
+                               "timed alone on a precomputed v",
+                     "kernel_us": kernel_ms * 1e3, "algorithmic_bytes_per_launch": alg_kernel},
+        "base_gemm_only": {"ms_per_step": base_ms, "note": "torch.matmul (cuBLAS) of x W^T alone, no delta"},
+        "unfused_layer": {"ms_per_step": unfused_ms, "value": job_value(T, world, unfused_ms),
+                          "note": "torch.matmul (cuBLAS) then lora_apply adding the delta to y in place"},
+        "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": total,
+                "d2h_bytes_per_step": T * d_out * 2},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, 1, args.cpu_seconds, layer=True)
     print(json.dumps(line), flush=True)
 
 

@@ -355,6 +355,19 @@ LORA_API int lora_linear(lora_pool *pool, int target, const void *x, int ldx, co
                 int ldw, void *y, int ldy, const int32_t *ids, const float *scales,
                 int T, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * The second half of lora_linear for callers that keep v = A_a x[t] (from
+ * lora_shrink): y[t] = bf16( W x[t] + scales[a] * B_a v[t, 0:r_a] ), one
+ * launch, no workspace.  v, ldv as lora_expand takes them (device fp32
+ * [T, ldv], ldv >= r_max, 4-byte aligned; rows without an adapter are not
+ * read); the other arguments as for lora_linear.  lora_shrink followed by
+ * lora_linear_expand gives y bit-identical to lora_linear.
+ */
+LORA_API int lora_linear_expand(lora_pool *pool, int target, const void *x, int ldx,
+                       const void *W, int ldw, const float *v, int ldv, void *y,
+                       int ldy, const int32_t *ids, const float *scales, int T,
+                       void *stream);
+
 /* Workspace of lora_linear for up to max_tokens rows on `target` (0 for bad
  * arguments). */
 LORA_API size_t lora_linear_workspace_bytes(const lora_pool *pool, int target, int max_tokens);

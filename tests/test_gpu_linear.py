@@ -172,3 +172,26 @@ def test_linear_rejects_bad_arguments(cuda_device):
             with pytest.raises(L.LoraError) as e:
                 fn()
             assert e.value.code == code
+
+
+@pytest.mark.parametrize("T", [64, 300])
+def test_shrink_then_linear_expand_equals_linear(cuda_device, T):
+    w = synth.custom(75 + T, T, [(512, 640)], [16, 8, 12, 16, 4, 16], 16)
+    with DevicePool(w, cuda_device) as pool:
+        dev = pool.device
+        x = to_dev_bf16(w.x(0), dev)
+        W = to_dev_bf16(w.W(0), dev)
+        ids = torch.from_numpy(w.ids).to(dev)
+        sc = torch.from_numpy(scales_of(w)).to(dev)
+        ws = _ws(pool, T)
+        y1 = torch.empty(T, 640, dtype=torch.bfloat16, device=dev)
+        y2 = torch.empty_like(y1)
+        L.lora_linear(pool.pool, 0, x, W, y1, ids, sc, ws)
+        v = torch.zeros(T, w.r_max + 8, dtype=torch.float32, device=dev)   # ldv past r_max
+        L.lora_shrink(pool.pool, 0, x, ids, v, ws)
+        n0 = L.lora_kernel_launches()
+        L.lora_linear_expand(pool.pool, 0, x, W, v, y2, ids, sc)
+        assert L.lora_kernel_launches() - n0 == 1
+        torch.cuda.synchronize(dev)
+        assert L.lora_get_error(pool.pool) == L.LORA_OK
+        assert np.array_equal(to_host_bits(y1), to_host_bits(y2))
