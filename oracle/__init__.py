@@ -22,6 +22,11 @@ Functions and the passages they follow (pages on multi-LoRA serving):
   formula (W stored d_out x d_in as in the column form W.x of "Serving Many
   LoRA Adapters From One Base Model", section "How it works"), and the whole
   layer output xW + (x A_i) B_i alpha/r.
+* ``moe_lora_apply`` -- the same per-row delta inside expert routing
+  ("Multi-LoRA Serving: Sharing One GPU Across Adapters", section "MoE Models
+  Raise the Bar": each adapted projection of every expert carries the
+  adapter's shrink and expand): every (token, chosen expert) pair takes the
+  delta of its own (adapter, expert) matrices.
 * ``group_rows``   -- "Multi-LoRA Serving: Why 100 Adapters Fit on One GPU",
   section "How does one batch run 30 different adapters at once?" (index
   vector, segmented gather).
@@ -204,6 +209,43 @@ def lora_linear(x, W, ids, n_slots: int, adapters: Adapters,
     (rows without a valid adapter get W x[t] alone).  Returns (y fp64, number
     of rows with an invalid id)."""
     return lora_apply(x, linear(x, W, threads), ids, n_slots, adapters, alpha, threads)
+
+
+def moe_pair_slots(lora_ids, topk_ids, n_experts: int, n_slots: int):
+    """Slot of each (token, chosen expert) pair, pair p = t * top_k + j:
+    lora_ids[t] * n_experts + topk_ids[t, j], or -1 when the token has no
+    adapter (lora_ids[t] == -1); an adapter id below -1, an expert outside
+    [0, n_experts) or a slot outside [0, n_slots) gives the invalid id
+    n_slots."""
+    lo = np.ascontiguousarray(lora_ids, dtype=np.int64)
+    tk = np.asarray(topk_ids, dtype=np.int64)
+    T, k = tk.shape
+    out = np.empty(T * k, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            a, e = int(lo[t]), int(tk[t, j])
+            if a == -1:
+                s = -1
+            elif a < -1 or e < 0 or e >= n_experts or a * n_experts + e >= n_slots:
+                s = n_slots
+            else:
+                s = a * n_experts + e
+            out[t * k + j] = s
+    return out.astype(np.int32)
+
+
+def moe_lora_apply(x, y_pairs, lora_ids, topk_ids, n_experts: int, n_slots: int,
+                   adapters: Adapters, alpha: Sequence[float], threads: int = 1):
+    """y_pairs[t * top_k + j] += (alpha_s / r_s) B_s (A_s x[t]) with s the
+    pair's slot (moe_pair_slots): the token's x row, the pair's own output row.
+    Returns (y_pairs fp64 [T * top_k, d_out], number of pairs with an invalid
+    id)."""
+    tk = np.asarray(topk_ids)
+    T, k = tk.shape
+    x64 = _as_f64(x)
+    x_pairs = np.repeat(x64, k, axis=0)           # row p holds x[p // top_k]
+    ids = moe_pair_slots(lora_ids, tk, n_experts, n_slots)
+    return lora_apply(x_pairs, y_pairs, ids, n_slots, adapters, alpha, threads)
 
 
 def group_rows(ids, n_slots: int, valid: Optional[np.ndarray] = None):

@@ -224,6 +224,61 @@ def test_lora_linear_without_adapters_is_the_base():
     assert bad == 0 and np.array_equal(y, oracle.linear(x, W))
 
 
+# ---------------------------------------------------------------- MoE pairs
+
+
+def test_moe_pair_slots_by_hand():
+    lora = np.array([1, -1, 0, 3, -2], np.int32)
+    topk = np.array([[2, 0], [1, 1], [3, 1], [0, 2], [1, 1]], np.int32)
+    got = oracle.moe_pair_slots(lora, topk, n_experts=4, n_slots=12)
+    # token 0: adapter 1 -> slots 6, 4; token 1: none; token 2: adapter 0 ->
+    # 3, 1; token 3: adapter 3 -> 12, 14 are past the 12 slots (invalid);
+    # token 4: adapter id -2 (invalid)
+    assert got.tolist() == [6, 4, -1, -1, 3, 1, 12, 12, 12, 12]
+
+
+def test_moe_integer_brute_force_exact():
+    g = np.random.default_rng(21)
+    T, k, E, n_ad, d_in, d_out = 5, 2, 3, 2, 4, 6
+    ranks = {}
+    adapters = {}
+    for a in range(n_ad):
+        for e in range(E):
+            r = int(g.integers(1, 4))
+            s = a * E + e
+            ranks[s] = r
+            adapters[s] = (g.integers(-2, 3, size=(r, d_in)).astype(np.float64),
+                           g.integers(-2, 3, size=(d_out, r)).astype(np.float64))
+    alpha = [2.0 * ranks[s] for s in range(n_ad * E)]
+    x = g.integers(-3, 4, size=(T, d_in)).astype(np.float64)
+    y = g.integers(-9, 10, size=(T * k, d_out)).astype(np.float64)
+    lora = np.array([0, 1, -1, 1, 0], np.int32)
+    topk = np.array([[0, 2], [1, 0], [2, 1], [2, 1], [1, 2]], np.int32)
+    got, bad = oracle.moe_lora_apply(x, y, lora, topk, E, n_ad * E, adapters, alpha)
+    assert bad == 0
+    for t in range(T):
+        for j in range(k):
+            p = t * k + j
+            for n in range(d_out):
+                ref = Fraction(int(y[p, n]))
+                if lora[t] >= 0:
+                    s = int(lora[t]) * E + int(topk[t, j])
+                    A, B = adapters[s]
+                    r = ranks[s]
+                    acc = Fraction(0)
+                    for q in range(r):
+                        acc += int(B[n, q]) * sum(int(x[t, c]) * int(A[q, c]) for c in range(d_in))
+                    ref += Fraction(int(alpha[s]), r) * acc
+                assert Fraction(got[p, n]) == ref, (t, j, n)
+
+
+def test_moe_one_expert_top1_is_the_plain_delta():
+    x, W, y_in, adapters, ids, alpha = _rand_case(22, 11, 16, 12, [3, 5], [6.0, 2.5])
+    got, bad = oracle.moe_lora_apply(x, y_in, ids, ids.reshape(-1, 1) * 0, 1, 2, adapters, alpha)
+    ref, bad2 = oracle.lora_apply(x, y_in, ids, 2, adapters, alpha)
+    assert bad == bad2 == 0 and np.array_equal(got, ref)
+
+
 def test_unit_vector_expand_is_a_column_of_B():
     # v = e_j  ->  delta = (alpha/r) * column j of B
     g = np.random.default_rng(7)
