@@ -89,6 +89,8 @@ _sig("lora_apply_segments", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _I, _P,
 _sig("lora_apply_multi", _I, [_P, _I, _P, _P, _I, _P, _I, _P, _P, _P, _I, _P, _Z, _P])
 _sig("lora_linear", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_linear_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
+_sig("lora_apply_moe", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _I, _I, _P, _P, _Z, _P])
+_sig("lora_moe_workspace_bytes", _Z, [_P, _I, _I])
 _sig("lora_shrink", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_noalloc", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
@@ -304,6 +306,20 @@ def lora_linear_expand(pool: PoolHandle, target: int, x, W, v, y, ids, scales, s
     _check(_lib.lora_linear_expand(pool, target, _ptr(x), _ld(x), _ptr(W), _ld(W), _ptr(v), _ld(v), _ptr(y),
                                    _ld(y), _ptr(ids), _ptr(scales), y.shape[0], _stream(stream)),
            "lora_linear_expand")
+
+
+def lora_moe_workspace_bytes(pool: PoolHandle, target: int, max_pairs: int) -> int:
+    return int(_lib.lora_moe_workspace_bytes(pool, target, max_pairs))
+
+
+def lora_apply_moe(pool: PoolHandle, target: int, x, y, lora_ids, topk_ids, n_experts: int, scales, ws,
+                   stream=None) -> None:
+    """Routed expert pairs: y[t * k + j] += s B_s (A_s x[t]), s = lora_ids[t] * n_experts + topk_ids[t, j];
+    x [T, d_in], y [T * k, d_out], topk_ids [T, k]."""
+    T, k = int(topk_ids.shape[0]), int(topk_ids.shape[1])
+    _check(_lib.lora_apply_moe(pool, target, _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(lora_ids), _ptr(topk_ids), T,
+                               k, n_experts, _ptr(scales), _ptr(ws), ws.numel(), _stream(stream)),
+           "lora_apply_moe")
 
 
 def lora_shrink(pool: PoolHandle, target: int, x, ids, v, ws, stream=None) -> None:

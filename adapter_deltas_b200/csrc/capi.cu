@@ -266,4 +266,44 @@ int lora_linear_expand(lora_pool *p, int target, const void *x, int ldx, const v
   return launch_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, v, ldv, T, static_cast<cudaStream_t>(stream));
 }
 
+size_t lora_moe_workspace_bytes(const lora_pool *p, int target, int max_pairs) {
+  if (!p || target < 0 || target >= p->n_targets || max_pairs < 0 || max_pairs > kMaxTokens) return 0;
+  return align256(plan_layout(max_pairs).total) + align256(size_t(max_pairs) * 4);
+}
+
+int lora_apply_moe(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const int32_t *lora_ids,
+                   const int32_t *topk_ids, int T, int top_k, int n_experts, const float *scales, void *ws,
+                   size_t ws_bytes, void *stream) {
+  if (!p || target < 0 || target >= p->n_targets || T < 0) return LORA_ERR_INVALID_ARG;
+  if (top_k < 1 || n_experts < 1 || (long long)T * top_k > kMaxTokens) return LORA_ERR_INVALID_ARG;
+  const int n_pairs = T * top_k;
+  int rc = check_call(p, target, n_pairs, ws, ws_bytes);
+  if (rc != LORA_OK || T == 0) return rc;
+  if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
+  if (!lora_ids || !topk_ids || !scales) return LORA_ERR_INVALID_ARG;
+  {
+    const char *xa = static_cast<const char *>(x), *ya = static_cast<const char *>(y);
+    if (xa < ya + size_t(n_pairs) * ldy * 2 && ya < xa + size_t(T) * ldx * 2) return LORA_ERR_INVALID_ARG;
+  }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_pairs <= kFusedMaxT) {
+    DeviceGuard g(p->device);
+    return launch_decode_moe(p, target, x, ldx, y, ldy, scales, lora_ids, topk_ids, n_pairs, top_k, n_experts,
+                             nullptr, st);
+  }
+  const size_t poff = align256(plan_layout(n_pairs).total);
+  if (ws_bytes < poff + size_t(n_pairs) * 4) return LORA_ERR_WORKSPACE;
+  int32_t *pair_ids = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + poff);
+  {
+    DeviceGuard g(p->device);
+    if ((rc = launch_moe_pair_ids(p, lora_ids, topk_ids, n_pairs, top_k, n_experts, pair_ids, st)) != LORA_OK)
+      return rc;
+  }
+  if ((rc = lora_plan_ids(p, pair_ids, n_pairs, ws, ws_bytes, stream)) != LORA_OK) return rc;
+  DeviceGuard g(p->device);
+  return launch_decode_moe(p, target, x, ldx, y, ldy, scales, lora_ids, topk_ids, n_pairs, top_k, n_experts, ws,
+                           st);
+}
+
 }  // extern "C"

@@ -328,6 +328,16 @@ int launch_decode_ids(lora_pool *pool, int mode, int target, const void *x, int 
 int launch_decode_multi(lora_pool *pool, int n_tgt, const int *targets, const int *y_cols, const void *x, int ldx,
                         void *y, int ldy, const float *scales, const int32_t *ids, int T, const void *ws,
                         cudaStream_t st);
+// Delta of routed expert pairs (pair p = token p / top_k, its (p % top_k)-th
+// expert; slot = adapter * n_experts + expert; x row p / top_k, y row p).
+// ws == nullptr: grouped in the kernel (n_pairs <= kFusedMaxT); else the plan
+// of the pairs' slots in ws.
+int launch_decode_moe(lora_pool *pool, int target, const void *x, int ldx, void *y, int ldy, const float *scales,
+                      const int32_t *lora_ids, const int32_t *topk, int n_pairs, int top_k, int n_experts,
+                      const void *ws, cudaStream_t st);
+// Writes each routed pair's slot (as launch_decode_moe forms it) to pair_ids.
+int launch_moe_pair_ids(const lora_pool *pool, const int32_t *lora_ids, const int32_t *topk, int n_pairs,
+                        int top_k, int n_experts, int32_t *pair_ids, cudaStream_t st);
 struct PrefillGeometry {
   int r_cap, kb_per, n_ks, n_stages, n_groups, smem_sh, smem_ex;
 };

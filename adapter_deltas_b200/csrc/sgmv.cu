@@ -62,6 +62,12 @@ struct DecodeArgs {
   int items_cap;  // entries the plan's items array has room for
   const int32_t *ids;  // non-null: group the rows of ids[0 .. T) inside the kernel (T <= kFusedMaxT)
   int T;
+  int x_div;           // row t reads x row t / x_div (1; top_k for routed expert pairs)
+  // routed expert pairs (moe_topk non-null, in-kernel grouping): row p is the
+  // pair (token p / moe_k, its (p % moe_k)-th expert), ids[] holds each
+  // token's adapter, and the pair's slot is adapter * moe_e + expert
+  const int32_t *moe_topk;
+  int moe_k, moe_e;
 };
 
 // ------------------------------------------------------------ warp MMA
@@ -350,12 +356,24 @@ __device__ __forceinline__ int slice_page(const PoolView &p, int slot, long long
   return pf == pl ? __ldg(p.pt + (long long)slot * p.pps + pf) : -1;
 }
 
+// Slot of routed pair p: -1 for a token without adapter; an adapter id below
+// -1, an expert outside [0, moe_e) or a slot past the pool gives n_slots
+// (reported as a bad id).
+__device__ __forceinline__ int moe_pair_slot(const DecodeArgs &a, int p) {
+  const int lo = a.ids[p / a.moe_k];
+  if (lo == -1) return -1;
+  const int e = a.moe_topk[p];
+  if (lo < -1 || e < 0 || e >= a.moe_e) return a.pool.n_slots;
+  const long long s = (long long)lo * a.moe_e + e;
+  return s < a.pool.n_slots ? (int)s : a.pool.n_slots;
+}
+
 __device__ int fused_plan(const DecodeArgs &a, const DecodeSmem &S, int tid, const SliceGeo &geo, int *any_bad) {
   const int T = a.T;
   int key = INT_MAX, bad = 0;
   int4 sinfo = make_int4(0, -1, -1, 0);
   if (tid < T) {
-    const int id = a.ids[tid];
+    const int id = a.moe_topk ? moe_pair_slot(a, tid) : a.ids[tid];
     if (id != -1) {
       if (id < -1 || id >= a.pool.n_slots) {
         bad = 1;
@@ -610,7 +628,7 @@ __global__ void __launch_bounds__(kDecodeThreads, JB >= 8 ? 1 : 2) decode_kernel
     is.wa1 = (unsigned long long)wa[1];
     is.wb0 = (unsigned long long)wb[0];
     is.wb1 = (unsigned long long)wb[1];
-    is.xrow = a.x ? (unsigned long long)(a.x + (long long)my_row * a.ldx + (long long)kv0 * 8) : 0ull;
+    is.xrow = a.x ? (unsigned long long)(a.x + (long long)(my_row / a.x_div) * a.ldx + (long long)kv0 * 8) : 0ull;
     is.yrow = a.y ? (unsigned long long)(a.y + (long long)my_row * a.ldy + a.y_col[ti] + (long long)nv0 * 8) : 0ull;
     ItemInfo &I = my_info[li % kItemSlots];
     if (lane < is.m) I.rows[lane] = my_row;
@@ -910,7 +928,8 @@ int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx,
 
 static int launch_decode_args(lora_pool *pool, int mode, int n_tgt, const int *targets, const int *y_cols,
                               const void *x, int ldx, void *y, int ldy, const float *scales, float *v, int ldv,
-                              int T, const void *ws, const int32_t *ids, cudaStream_t st, int items_hdr) {
+                              int T, const void *ws, const int32_t *ids, cudaStream_t st, int items_hdr,
+                              int x_div = 1, const int32_t *moe_topk = nullptr, int moe_k = 0, int moe_e = 0) {
   DecodeArgs a;
   a.pool = pool->view();
   a.d_in = pool->targets[targets[0]].d_in;
@@ -943,6 +962,10 @@ static int launch_decode_args(lora_pool *pool, int mode, int n_tgt, const int *t
   a.items_cap = ids ? 0 : plan_layout(T).i_max;
   a.ids = ids;
   a.T = T;
+  a.x_div = x_div;
+  a.moe_topk = moe_topk;
+  a.moe_k = moe_k;
+  a.moe_e = moe_e;
   a.v = v;
   a.ldv = ldv;
   a.status = pool->d_status;
@@ -995,6 +1018,19 @@ int launch_decode_ids(lora_pool *pool, int mode, int target, const void *x, int 
   if (T < 1 || T > kFusedMaxT) return LORA_ERR_INVALID_ARG;
   return launch_decode_args(pool, mode, 1, &target, nullptr, x, ldx, y, ldy, scales, v, ldv, T, nullptr, ids, st,
                             kHdrItems);
+}
+
+int launch_decode_moe(lora_pool *pool, int target, const void *x, int ldx, void *y, int ldy, const float *scales,
+                      const int32_t *lora_ids, const int32_t *topk, int n_pairs, int top_k, int n_experts,
+                      const void *ws, cudaStream_t st) {
+  if (!ws) {  // pairs grouped inside the kernel from the routing itself
+    if (n_pairs < 1 || n_pairs > kFusedMaxT) return LORA_ERR_INVALID_ARG;
+    return launch_decode_args(pool, kFused, 1, &target, nullptr, x, ldx, y, ldy, scales, nullptr, 0, n_pairs,
+                              nullptr, lora_ids, st, kHdrItems, top_k, topk, top_k, n_experts);
+  }
+  // the pairs' slots were planned into ws (lora_plan_ids over them)
+  return launch_decode_args(pool, kFused, 1, &target, nullptr, x, ldx, y, ldy, scales, nullptr, 0, n_pairs, ws,
+                            nullptr, st, kHdrItems, top_k);
 }
 
 int launch_decode_multi(lora_pool *pool, int n_tgt, const int *targets, const int *y_cols, const void *x, int ldx,

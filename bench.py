@@ -1,7 +1,7 @@
 """Benchmark of the multi-LoRA delta path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload q_proj|tiny|prefill|mlp|paged|qkv|swapin|linear]
+                    [--workload q_proj|tiny|prefill|mlp|paged|qkv|swapin|linear|moe]
 
 Default workload (the metric's configuration): Llama-2-7B q_proj-shaped decode,
 d_in = d_out = 4096, rank 16 for all, 32 resident adapters in a contiguous
@@ -43,8 +43,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "LoRA-delta tokens/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
-WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5, "qkv": 2, "swapin": 5, "linear": 2}
+WORKLOADS = {"tiny": 1, "q_proj": 2, "prefill": 3, "mlp": 4, "paged": 5, "qkv": 2, "swapin": 5, "linear": 2,
+             "moe": 2}
 LINEAR_WORKLOAD = "q_proj layer with its delta fused: y = x W^T + delta, d4096 r16 32 adapters 64 tokens"
+MOE_WORKLOAD = ("routed expert pairs: 64 tokens x top-4 of 32 experts, 8 adapters (256 slots), rank 16, "
+                "expert projection 2880 -> 2880")
+MOE_SHAPE = dict(T=64, k=4, E=32, n_ad=8, d=2880, r=16)
 L2_BYTES = 126 * 2 ** 20
 FUSED_MAX_T = 256   # batches up to this size are grouped inside the decode kernel (one launch)
 
@@ -187,6 +191,8 @@ def run_reference(args, rank: int, world: int):
     is scaled by their count."""
     if rank != 0:
         return
+    if args.workload == "moe":
+        return run_reference_moe(args)
     import synth
     w = synth.config(WORKLOADS[args.workload])
     n_t = len(w.targets) if args.workload == "paged" else 3 if args.workload == "qkv" else 1
@@ -208,6 +214,23 @@ def run_reference(args, rank: int, world: int):
         "config": {"workload": LINEAR_WORKLOAD if args.workload == "linear" else w.name, "global_batch": w.T,
                    "seq_len": 1, "parallelism": "oracle on host cores"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_moe(args):
+    """The oracle on the routed-pair workload: warm-up calls, then K timed."""
+    moe_cpu_baseline(0.0, max_calls=args.warmup)
+    cb = moe_cpu_baseline(0.0, max_calls=args.steps)
+    value = cb["value"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * MOE_SHAPE["T"] / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": MOE_WORKLOAD, "global_batch": MOE_SHAPE["T"], "seq_len": 1,
+                   "parallelism": "oracle on host cores"},
+        "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -255,6 +278,8 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         return run_swapin(args, rank, world, dev, bf16)
     if args.workload == "linear":
         return run_linear(args, rank, world, dev, w, scales, bf16)
+    if args.workload == "moe":
+        return run_moe(args, rank, world, dev, bf16)
 
     # one buffer set: pool (all slots loaded), x, y, ids, workspace
     pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
@@ -820,6 +845,158 @@ def run_linear(args, rank, world, dev, w, scales, bf16):
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(w, 1, args.cpu_seconds, layer=True)
     print(json.dumps(line), flush=True)
+
+
+def moe_workload(seed: int):
+    """The routed workload: a synth pool of n_ad * E slots (adapter a's
+    matrices for expert e in slot a * E + e), each token's adapter uniform
+    over the adapters (10 % none) and top_k distinct experts per token."""
+    import synth
+    m = MOE_SHAPE
+    w = synth.custom(seed, m["T"], [(m["d"], m["d"])], [m["r"]] * (m["n_ad"] * m["E"]), m["r"])
+    g = np.random.default_rng(seed + 1)
+    lora = g.integers(0, m["n_ad"], size=m["T"]).astype(np.int32)
+    lora[g.permutation(m["T"])[:round(0.1 * m["T"])]] = -1
+    topk = np.stack([g.permutation(m["E"])[:m["k"]] for _ in range(m["T"])]).astype(np.int32)
+    y = synth.normal_bf16(np.random.default_rng(seed + 2), (m["T"] * m["k"], m["d"]), 1.0)
+    return w, lora, topk, y
+
+
+def run_moe(args, rank, world, dev, bf16):
+    """The delta inside expert routing: one lora_apply_moe per step over the
+    256 (token, expert) pairs of 64 tokens routed to 4 of 32 experts, each
+    pair taking its own (adapter, expert) slot (one launch: the pairs' slots
+    are formed and grouped inside the delta kernel)."""
+    import torch
+
+    import adapter_deltas_b200 as L
+    m = MOE_SHAPE
+    w, lora, topk, y_np = moe_workload(4000 + rank)
+    T, k, E, d = m["T"], m["k"], m["E"], m["d"]
+    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, 0)
+    set_bytes = pool_bytes + (T * d + T * k * d) * 2
+    n_sets = max(2, min(32, -(-4 * L2_BYTES // set_bytes)))
+    w.prefetch(range(w.n_slots), [0])
+    adapters = {s_: tuple(bf16(t) for t in w.adapter(s_, 0)) for s_ in range(w.n_slots)}
+    sc_np = (w.alpha / w.rank).astype(np.float32)
+    scales = torch.from_numpy(sc_np).to(dev)
+    x0, y0 = bf16(w.x(0)), bf16(y_np)
+    lo0, tk0 = torch.from_numpy(lora).to(dev), torch.from_numpy(topk).to(dev)
+    sets = []
+    for _ in range(n_sets):
+        mem = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
+        pool = L.lora_pool_create(dev.index, w.targets, w.r_max, w.n_slots, 0, mem, 0)
+        for s_, (A, B) in adapters.items():
+            L.lora_pool_load(pool, s_, 0, int(w.rank[s_]), A, B)
+        sets.append(dict(pool=pool, mem=mem, x=x0.clone(), y=y0.clone(), lo=lo0.clone(), tk=tk0.clone(),
+                         ws=torch.zeros(max(256, L.lora_moe_workspace_bytes(pool, 0, T * k)), dtype=torch.uint8,
+                                        device=dev)))
+    torch.cuda.synchronize()
+
+    def step(i):
+        s_ = sets[i % n_sets]
+        L.lora_apply_moe(s_["pool"], 0, s_["x"], s_["y"], s_["lo"], s_["tk"], E, scales, s_["ws"])
+
+    def timed(fn, n):
+        g_w, _ = capture_graph(dev, fn, range(args.warmup))
+        g, launches = capture_graph(dev, fn, range(n))
+        g_w.replay()
+        torch.cuda.synchronize()
+        sync_ranks(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        g.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        sync_ranks(world)
+        del g, g_w
+        return reduce_max(ev0.elapsed_time(ev1) / n, world, dev), launches
+
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        ms, launches = timed(step, args.steps)
+    clocks = sampler.stop()
+
+    # end to end: x, adapter ids and routing in from one packed pinned buffer,
+    # the pairs' output rows in and out, every step
+    parts = [lo0.cpu().view(torch.uint8), tk0.cpu().view(torch.uint8).reshape(-1),
+             x0.cpu().view(torch.uint8).reshape(-1), y0.cpu().view(torch.uint8).reshape(-1)]
+    offs, total = [], 0
+    for t_ in parts:
+        offs.append(total)
+        total += -(-t_.numel() // 256) * 256
+    packed_h = torch.zeros(total, dtype=torch.uint8).pin_memory()
+    for o, t_ in zip(offs, parts):
+        packed_h[o:o + t_.numel()] = t_
+    yout = torch.empty(T * k, d, dtype=torch.bfloat16).pin_memory()
+    packed_d = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(n_sets)]
+
+    def e2e_step(i):
+        s_ = sets[i % n_sets]
+        buf = packed_d[i % n_sets]
+        buf.copy_(packed_h, non_blocking=True)
+        lo = buf[offs[0]:offs[0] + T * 4].view(torch.int32)
+        tk = buf[offs[1]:offs[1] + T * k * 4].view(torch.int32).view(T, k)
+        x = buf[offs[2]:offs[2] + T * d * 2].view(torch.bfloat16).view(T, d)
+        y = buf[offs[3]:offs[3] + T * k * d * 2].view(torch.bfloat16).view(T * k, d)
+        L.lora_apply_moe(s_["pool"], 0, x, y, lo, tk, E, scales, s_["ws"])
+        yout.copy_(y, non_blocking=True)
+
+    e2e_ms, _ = timed(e2e_step, args.steps)
+    for s_ in sets:
+        L.lora_pool_destroy(s_["pool"])
+    if rank != 0:
+        return
+    peak, peak_kind = load_peaks()
+    import oracle
+    slots = oracle.moe_pair_slots(lora, topk, E, w.n_slots)
+    act = slots[slots >= 0]
+    distinct = np.unique(act)
+    # each distinct slot's A and B, the adapted tokens' x once, the adapted
+    # pairs' y read and written
+    alg = (int(sum(int(w.rank[s_]) * 2 * d * 2 for s_ in distinct)) + int((lora >= 0).sum()) * d * 2
+           + act.size * d * 4)
+    achieved = alg / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": job_value(T, world, ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": MOE_WORKLOAD, "global_batch": T * world, "seq_len": 1,
+                   "parallelism": "replicas%d" % world if world > 1 else "single",
+                   "pairs": T * k, "slots_in_batch": int(distinct.size),
+                   "l2": "%d rotating buffer sets, %.0f MB > 4x L2" % (n_sets, n_sets * set_bytes / 1e6),
+                   "timing": "CUDA graph of the K steps, CUDA events around its replay"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "decode_kernel<fused> forming and grouping the pairs' slots in-kernel (the whole step)",
+                     "kernel_us": ms * 1e3, "algorithmic_bytes_per_launch": alg},
+        "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": total,
+                "d2h_bytes_per_step": T * k * d * 2},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if world == 1:
+        line["cpu_baseline"] = moe_cpu_baseline(args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def moe_cpu_baseline(seconds: float, max_calls: int = 1 << 30):
+    """The oracle's routed-pair delta on the host cores, whole batches."""
+    import oracle
+    m = MOE_SHAPE
+    w, lora, topk, y = moe_workload(4000)
+    slots = oracle.moe_pair_slots(lora, topk, m["E"], w.n_slots)
+    adapters = {int(s_): w.adapter(int(s_), 0) for s_ in np.unique(slots[slots >= 0])}
+    threads = min(cpu_threads(), m["T"] * m["k"])
+    x = w.x(0)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.moe_lora_apply(x, y, lora, topk, m["E"], w.n_slots, adapters, w.alpha, threads=threads)
+        n += 1
+        el = time.perf_counter() - t0
+        if (seconds > 0 and el >= seconds) or n >= max_calls:
+            break
+    return {"value": n * m["T"] / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d whole batches of %d tokens (%d pairs) (%.1f s)" % (n, m["T"], m["T"] * m["k"], el)}
 
 
 def run_swapin(args, rank, world, dev, bf16):

@@ -324,6 +324,43 @@ LORA_API int lora_apply_multi(lora_pool *pool, int n_targets, const int *targets
                      const int32_t *ids, const float *scales, int T, void *ws,
                      size_t ws_bytes, void *stream);
 
+/* ------------------------------------------------ routed expert pairs */
+
+/*
+ * The delta inside expert routing (mixture-of-experts layers): each token t
+ * is routed to top_k experts, and an adapted expert projection carries the
+ * token's adapter's own shrink and expand for that expert ("Multi-LoRA
+ * Serving: Sharing One GPU Across Adapters", section "MoE Models Raise the
+ * Bar").  For every pair p = t * top_k + j:
+ *     y[p] += scales[s] * B_s (A_s x[t]),  s = lora_ids[t] * n_experts + topk_ids[p],
+ * with slot s of the pool holding adapter lora_ids[t]'s matrices for expert
+ * topk_ids[p] on `target`.
+ *   x, ldx     device bf16 [T, ldx]: one row per token
+ *   y, ldy     device bf16 [T * top_k, ldy]: one row per pair (the expert
+ *              output rows, in pair order), updated in place
+ *   lora_ids   device int32 [T]: the token's adapter, -1 = none (its pairs'
+ *              rows are untouched)
+ *   topk_ids   device int32 [T * top_k]: the experts chosen for each token
+ *   n_experts  experts per adapter (slots are adapter * n_experts + expert)
+ *   scales, ws, ws_bytes, stream  as for lora_apply, with
+ *              lora_moe_workspace_bytes(T * top_k)
+ * Up to 256 pairs take one launch (the slots are formed and grouped inside
+ * the delta kernel); beyond, three (pair slots, plan, delta).  A token's
+ * adapter id below -1, an expert outside [0, n_experts) or a slot past the
+ * pool raises the sticky LORA_ERR_BAD_ID and leaves that pair's row
+ * untouched; an empty slot raises LORA_ERR_NOT_LOADED.  Equal, bit for bit,
+ * to lora_apply on x with each token's row repeated top_k times and ids set
+ * to the pairs' slots.
+ */
+LORA_API int lora_apply_moe(lora_pool *pool, int target, const void *x, int ldx, void *y,
+                   int ldy, const int32_t *lora_ids, const int32_t *topk_ids, int T,
+                   int top_k, int n_experts, const float *scales, void *ws,
+                   size_t ws_bytes, void *stream);
+
+/* Workspace of lora_apply_moe for up to max_pairs (T * top_k) pairs on
+ * `target` (0 for bad arguments). */
+LORA_API size_t lora_moe_workspace_bytes(const lora_pool *pool, int target, int max_pairs);
+
 /* ------------------------------------------ the layer with its delta fused */
 
 /*
