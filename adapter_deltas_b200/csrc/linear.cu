@@ -12,8 +12,8 @@
 //
 // Two launches.  The decode kernel in shrink mode writes v = A_a x[t] (fp32)
 // for every adapted row; then this kernel, launched as its programmatic
-// dependent (it streams W and x while the shrink still runs, and only the
-// delta waits for v):
+// dependent (only the delta waits for v; the W stream may start while the
+// shrink still runs, where an SM has room for both):
 //   tile     = 128 output features (MMA M) x NT rows of the batch (MMA N).
 //              The features are the A operand (W rows, K-major), so a decode
 //              batch of 16 .. 256 rows is the N of a single MMA.
@@ -22,7 +22,9 @@
 //              then, as further K steps of the same TMEM accumulator, its
 //              share of the tile's adapters (adapter index mod split):
 //                D[f, t] += sum_j B_a^T[j, f] (s_a v[t, j])  (rows of adapter a only)
-//              with s_a v split into two bf16 terms (hi + lo, ~16 bits kept).
+//              with s_a v split into two bf16 terms (hi + lo, ~16 bits kept),
+//              16 ranks per chunk, chunks resident in shared memory in groups
+//              (the first group's B^T slices load during the W stream).
 //   epilogue = the split partials meet in the owning CTA's shared memory
 //              (DSMEM stores between two cluster barriers), are summed in
 //              fixed order and rounded to bf16 once.
