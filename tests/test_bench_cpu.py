@@ -1,7 +1,8 @@
 """Host-side helpers of bench.py: the ncu traffic figure is read from a
 profile summary only while its source hash matches the kernel source, and the
 algorithmic bytes follow the definition (distinct adapters at their own rank,
-x of the adapted rows, y of the adapted rows read and written)."""
+x of the adapted rows, y of the adapted rows read and written), and the routed
+workload draws valid routing."""
 
 import hashlib
 import os
@@ -38,3 +39,20 @@ def test_algorithmic_bytes_definition():
     # adapted rows: ids 0, 1, 1, 0 (slot 2 has rank 0: not adapted)
     want = (8 + 16) * (64 + 32) * 2 + 4 * 64 * 2 + 4 * 32 * 4
     assert bench.algorithmic_bytes(w, 0, np.asarray(w.ids)) == want
+
+
+def test_moe_workload_routing():
+    # every token picks top_k distinct experts; 10 % of tokens carry no
+    # adapter; the pool has one slot per (adapter, expert); output rows per pair
+    m = bench.MOE_SHAPE
+    w, lora, topk, y = bench.moe_workload(4000)
+    assert w.n_slots == m["n_ad"] * m["E"] and w.targets == [(m["d"], m["d"])]
+    assert w.x(0).shape == (m["T"], m["d"])
+    assert topk.shape == (m["T"], m["k"]) and y.shape == (m["T"] * m["k"], m["d"])
+    assert all(len(set(row)) == m["k"] for row in topk.tolist())
+    assert topk.min() >= 0 and topk.max() < m["E"]
+    assert (lora == -1).sum() == round(0.1 * m["T"])
+    assert lora.max() < m["n_ad"] and lora.min() >= -1
+    # seeded: the same seed gives the same routing
+    _, lora2, topk2, _ = bench.moe_workload(4000)
+    assert np.array_equal(lora, lora2) and np.array_equal(topk, topk2)
