@@ -967,7 +967,9 @@ def run_moe(args, rank, world, dev, bf16):
                    "l2": "%d rotating buffer sets, %.0f MB > 4x L2" % (n_sets, n_sets * set_bytes / 1e6),
                    "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": None,
+                     "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "sgmv.cu", "moe"),
+                     "traffic_note": "DRAM bytes of one launch from the ncu summary in profiles/, while its "
+                                     "source hash matches",
                      "kernel": "decode_kernel<fused> forming and grouping the pairs' slots in-kernel (the whole step)",
                      "kernel_us": ms * 1e3, "algorithmic_bytes_per_launch": alg},
         "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": total,
