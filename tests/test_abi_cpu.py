@@ -92,3 +92,16 @@ def test_workspace_and_plan_layout_need_no_device(L):
     assert lib.lora_workspace_bytes(None, 0, 64) == 0
     assert lib.lora_apply(None, 0, None, 0, None, 0, None, None, 4, None, 0, None) == L.LORA_ERR_INVALID_ARG
     assert L.lora_kernel_launches() == 0
+
+
+def test_layer_and_routed_calls_reject_a_null_pool_without_device_work(L):
+    lib = L._lib
+    assert lib.lora_linear_workspace_bytes(None, 0, 64) == 0
+    assert lib.lora_moe_workspace_bytes(None, 0, 64) == 0
+    n0 = L.lora_kernel_launches()
+    assert lib.lora_linear(None, 0, None, 0, None, 0, None, 0, None, None, 4, None, 0, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_linear_expand(None, 0, None, 0, None, 0, None, 0, None, 0, None, None, 4,
+                                  None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_apply_moe(None, 0, None, 0, None, 0, None, None, 4, 2, 8, None, None, 0,
+                              None) == L.LORA_ERR_INVALID_ARG
+    assert L.lora_kernel_launches() == n0
