@@ -50,7 +50,7 @@ class lora_target(ctypes.Structure):
 class lora_pool_info(ctypes.Structure):
     _fields_ = [("slot_bytes", _Z), ("page_bytes", _Z), ("pages_per_slot", _I), ("n_pages", _I),
                 ("free_pages", _I), ("n_slots", _I), ("n_targets", _I), ("r_max", _I),
-                ("decode_clusters", _I)]
+                ("decode_ctas", _I)]
 
 
 class lora_plan_layout(ctypes.Structure):
@@ -96,6 +96,7 @@ _sig("lora_expand", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_noalloc", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
 _sig("lora_get_error", _I, [_P, ctypes.POINTER(_I), _P])
 _sig("lora_kernel_launches", ctypes.c_uint64, [])
+_sig("lora_set_wait_limit_ns", None, [ctypes.c_uint64])
 
 
 class LoraError(RuntimeError):
@@ -336,7 +337,7 @@ LORA_NOALLOC_MAX_TOKENS = 4096
 
 
 def lora_apply_noalloc(pool: PoolHandle, target: int, x, y, ids, scales, stream=None) -> None:
-    """lora_apply without a workspace argument: the plan lives in a fixed
+    """lora_apply without a workspace argument: the workspace lives in a fixed
     device array inside the library (for callers that cannot allocate).
     Calls that overlap on the GPU share that array and must be serialised."""
     _check(_lib.lora_apply_noalloc(pool, target, _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(ids), _ptr(scales),
@@ -351,3 +352,8 @@ def lora_get_error(pool: PoolHandle, stream=None) -> int:
 
 def lora_kernel_launches() -> int:
     return int(_lib.lora_kernel_launches())
+
+
+def lora_set_wait_limit_ns(ns: int) -> None:
+    """Wall-clock limit of the decode kernel's bounded waits (0: one second)."""
+    _lib.lora_set_wait_limit_ns(int(ns))

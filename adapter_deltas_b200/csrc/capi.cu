@@ -92,6 +92,8 @@ int lora_plan_layout_get(const lora_pool *p, int T, lora_plan_layout *out) {
 
 int lora_mma_min_rows(void) { return kMmaMinRows; }
 
+void lora_set_wait_limit_ns(uint64_t ns) { set_wait_limit_ns(ns); }
+
 int lora_plan_ids(lora_pool *p, const int32_t *ids, int T, void *ws, size_t ws_bytes, void *stream) {
   int rc = check_call(p, 0, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
@@ -126,17 +128,27 @@ int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, i
   DeviceGuard g(p->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int kind = plan_kind(p, ws);
+  DecodeCall c;
+  c.targets = &target;
+  c.x = x;
+  c.ldx = ldx;
+  c.y = y;
+  c.ldy = ldy;
+  c.scales = scales;
+  c.T = T;
+  c.ws = const_cast<void *>(ws);
   if (kind == kPlanIds)  // index-vector plans hold decode items only
-    return launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItems);
+    return launch_decode(p, c, st);
   PrefillGeometry geo;
   if (kind == kPlanSegments && prefill_geometry(p, target, plan_layout(T).j_max, &geo)) {
     // short segments on the decode kernel, long ones on the tensor cores
-    rc = launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItems);
+    rc = launch_decode(p, c, st);
     if (rc != LORA_OK) return rc;
     return launch_prefill(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, st);
   }
   // every segment on the decode kernel
-  return launch_decode_items(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, T, ws, st, kHdrItemsAll);
+  c.items_hdr = kHdrItemsAll;
+  return launch_decode(p, c, st);
 }
 
 int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const int32_t *ids,
@@ -149,8 +161,17 @@ int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ld
   if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
   if (T <= kFusedMaxT) {  // one launch: the delta kernel groups the rows itself
     DeviceGuard g(p->device);
-    return launch_decode_ids(p, kFused, target, x, ldx, y, ldy, scales, nullptr, 0, ids, T,
-                             static_cast<cudaStream_t>(stream));
+    DecodeCall c;
+    c.targets = &target;
+    c.x = x;
+    c.ldx = ldx;
+    c.y = y;
+    c.ldy = ldy;
+    c.scales = scales;
+    c.T = T;
+    c.ws = ws;
+    c.ids = ids;
+    return launch_decode(p, c, static_cast<cudaStream_t>(stream));
   }
   if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
   return lora_apply_plan(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, stream);
@@ -177,13 +198,25 @@ int lora_apply_multi(lora_pool *p, int n_targets, const int *targets, const void
   if (!scales || !ids) return LORA_ERR_INVALID_ARG;
   if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DecodeCall c;
+  c.n_tgt = n_targets;
+  c.targets = targets;
+  c.y_cols = y_cols;
+  c.x = x;
+  c.ldx = ldx;
+  c.y = y;
+  c.ldy = ldy;
+  c.scales = scales;
+  c.T = T;
+  c.ws = ws;
   if (T <= kFusedMaxT) {
     DeviceGuard g(p->device);
-    return launch_decode_multi(p, n_targets, targets, y_cols, x, ldx, y, ldy, scales, ids, T, nullptr, st);
+    c.ids = ids;
+    return launch_decode(p, c, st);
   }
   if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
   DeviceGuard g(p->device);
-  return launch_decode_multi(p, n_targets, targets, y_cols, x, ldx, y, ldy, scales, nullptr, T, ws, st);
+  return launch_decode(p, c, st);
 }
 
 int lora_apply_segments(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
@@ -206,15 +239,23 @@ int lora_shrink(lora_pool *p, int target, const void *x, int ldx, const int32_t 
   if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
   if (!ids || !v || ldv < p->r_max) return LORA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(v) & 3u) return LORA_ERR_ALIGNMENT;
+  DecodeCall c;
+  c.mode = kShrinkOnly;
+  c.targets = &target;
+  c.x = x;
+  c.ldx = ldx;
+  c.v = v;
+  c.ldv = ldv;
+  c.T = T;
+  c.ws = ws;
   if (T <= kFusedMaxT) {
     DeviceGuard g(p->device);
-    return launch_decode_ids(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, ldv, ids, T,
-                             static_cast<cudaStream_t>(stream));
+    c.ids = ids;
+    return launch_decode(p, c, static_cast<cudaStream_t>(stream));
   }
   if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
   DeviceGuard g(p->device);
-  return launch_decode(p, kShrinkOnly, target, x, ldx, nullptr, 0, nullptr, v, ldv, T, ws,
-                       static_cast<cudaStream_t>(stream));
+  return launch_decode(p, c, static_cast<cudaStream_t>(stream));
 }
 
 int lora_expand(lora_pool *p, int target, const float *v, int ldv, void *y, int ldy, const int32_t *ids,
@@ -224,15 +265,24 @@ int lora_expand(lora_pool *p, int target, const float *v, int ldv, void *y, int 
   if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
   if (!ids || !v || !scales || ldv < p->r_max) return LORA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(v) & 3u) return LORA_ERR_ALIGNMENT;
+  DecodeCall c;
+  c.mode = kExpandOnly;
+  c.targets = &target;
+  c.y = y;
+  c.ldy = ldy;
+  c.scales = scales;
+  c.v = const_cast<float *>(v);
+  c.ldv = ldv;
+  c.T = T;
+  c.ws = ws;
   if (T <= kFusedMaxT) {
     DeviceGuard g(p->device);
-    return launch_decode_ids(p, kExpandOnly, target, nullptr, 0, y, ldy, scales, const_cast<float *>(v), ldv, ids,
-                             T, static_cast<cudaStream_t>(stream));
+    c.ids = ids;
+    return launch_decode(p, c, static_cast<cudaStream_t>(stream));
   }
   if ((rc = lora_plan_ids(p, ids, T, ws, ws_bytes, stream)) != LORA_OK) return rc;
   DeviceGuard g(p->device);
-  return launch_decode(p, kExpandOnly, target, nullptr, 0, y, ldy, scales, const_cast<float *>(v), ldv, T, ws,
-                       static_cast<cudaStream_t>(stream));
+  return launch_decode(p, c, static_cast<cudaStream_t>(stream));
 }
 
 size_t lora_linear_workspace_bytes(const lora_pool *p, int target, int max_tokens) {
@@ -287,10 +337,23 @@ int lora_apply_moe(lora_pool *p, int target, const void *x, int ldx, void *y, in
     if (xa < ya + size_t(n_pairs) * ldy * 2 && ya < xa + size_t(T) * ldx * 2) return LORA_ERR_INVALID_ARG;
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (n_pairs <= kFusedMaxT) {
+  DecodeCall c;
+  c.targets = &target;
+  c.x = x;
+  c.ldx = ldx;
+  c.y = y;
+  c.ldy = ldy;
+  c.scales = scales;
+  c.T = n_pairs;
+  c.ws = ws;
+  c.x_div = top_k;
+  if (n_pairs <= kFusedMaxT) {  // pairs grouped inside the kernel from the routing itself
     DeviceGuard g(p->device);
-    return launch_decode_moe(p, target, x, ldx, y, ldy, scales, lora_ids, topk_ids, n_pairs, top_k, n_experts,
-                             nullptr, st);
+    c.ids = lora_ids;
+    c.moe_topk = topk_ids;
+    c.moe_k = top_k;
+    c.moe_e = n_experts;
+    return launch_decode(p, c, st);
   }
   const size_t poff = align256(plan_layout(n_pairs).total);
   if (ws_bytes < poff + size_t(n_pairs) * 4) return LORA_ERR_WORKSPACE;
@@ -302,8 +365,7 @@ int lora_apply_moe(lora_pool *p, int target, const void *x, int ldx, void *y, in
   }
   if ((rc = lora_plan_ids(p, pair_ids, n_pairs, ws, ws_bytes, stream)) != LORA_OK) return rc;
   DeviceGuard g(p->device);
-  return launch_decode_moe(p, target, x, ldx, y, ldy, scales, lora_ids, topk_ids, n_pairs, top_k, n_experts, ws,
-                           st);
+  return launch_decode(p, c, st);  // the pairs' slots were planned into ws
 }
 
 }  // extern "C"

@@ -29,12 +29,9 @@ constexpr int kItemRows = 16;        // rows per decode work item
 constexpr int kMmaRows = 128;        // rows per tensor-core tile
 constexpr int kMmaMinRows = 64;     // segment length that selects the tensor-core path
 constexpr int kPlanThreads = 1024;
-constexpr int kConsumerWarps = 8;    // decode kernel: 8 warps, each copies and computes
+constexpr int kConsumerWarps = 8;    // decode kernel: 8 compute warps (plus one producer warp)
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kDecodeThreads = kConsumerThreads;
-constexpr int kClusterCtas = 8;      // CTAs that split one work item (portable cluster)
 constexpr int kMaxStages = 4;        // barrier slots of the decode ring (it runs n_stages <= this)
-constexpr int kItemSlots = 8;        // items a warp's copies may run ahead of its compute
 constexpr int kFusedMaxT = 256;      // batches up to this size are grouped inside the decode kernel
 constexpr int kMaxMulti = 4;         // targets sharing x in one decode launch
 
@@ -72,17 +69,56 @@ __device__ __forceinline__ const uint8_t *pool_addr(const PoolView &p, int slot,
   return p.base + (long long)phys * p.page_bytes + inside;
 }
 
+// Physical page holding a slot's whole block [first, first + bytes), or -1
+// when the block spans pages (its pieces are then located one by one).
+__device__ __forceinline__ int block_page(const PoolView &p, int slot, long long first, long long bytes) {
+  if (p.log2_page < 0) return __ldg(p.pt + (long long)slot * p.pps);
+  const long long pf = first >> p.log2_page, pl = (first + bytes - 1) >> p.log2_page;
+  return pf == pl ? __ldg(p.pt + (long long)slot * p.pps + pf) : -1;
+}
+
+// Address of logical byte `off` of a slot whose block lies on physical page
+// `page` (block_page >= 0).
+__device__ __forceinline__ const uint8_t *page_addr(const PoolView &p, int page, long long off) {
+  return p.base + (long long)page * p.page_bytes + (p.log2_page < 0 ? off : (off & (p.page_bytes - 1)));
+}
+
+// Arrangement of an adapter block inside a slot.  A block (A: r_max rows of
+// d_in bf16; B^T: r_max rows of d_out bf16) is stored in column tiles of
+// pool_tile_cols(r_max) columns (32 KiB of r_max rows) -- the tile the decode
+// kernel stages with one bulk copy.  Tile k holds columns [k * tc, min((k + 1) * tc, width)) of rows
+// 0 .. r_max - 1, one row after the other, so the first r rows of a tile are
+// one contiguous range.  Inside a row of a tile, the 16-byte chunks of every
+// complete group of eight are permuted, chunk c stored at c ^ (row % 8) (a
+// trailing partial group keeps its order): the rows of a staged tile then
+// sit in different shared-memory banks for the MMA operand loads.
+__host__ __device__ constexpr int pool_tile_cols(int r_max) { return r_max <= 16 ? 1024 : r_max <= 32 ? 512 : 256; }
+
+__host__ __device__ constexpr int swz_chunk(int c, int row, int chunks) {
+  return ((c | 7) < chunks) ? (c ^ (row & 7)) : c;
+}
+
+// Byte offset, inside a block of `width` columns, of 16-byte chunk `chunk`
+// (columns 8 chunk .. 8 chunk + 7) of row `row`.
+__host__ __device__ constexpr long long block_chunk_off(int row, int chunk, int width, int r_max) {
+  const int tcc = pool_tile_cols(r_max) / 8;  // chunks per full tile
+  const int k = chunk / tcc, c = chunk - k * tcc;
+  const int rest = width / 8 - k * tcc;
+  const int tw = rest < tcc ? rest : tcc;  // chunks in this tile
+  return (long long)k * r_max * tcc * 16 + (long long)row * tw * 16 + (long long)swz_chunk(c, row, tw) * 16;
+}
+
 // Plan arrays inside the workspace (byte offsets from its base).
 struct PlanLayout {
   size_t header, perm, seg_start, seg_slot, seg_row, items, tiles, total;
   int s_max, i_max, j_max;
 };
 
-inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline PlanLayout plan_layout(int T) {
-  PlanLayout L;
-  int t = T > 0 ? T : 1;
+constexpr PlanLayout plan_layout(int T) {
+  PlanLayout L{};
+  const int t = T > 0 ? T : 1;
   L.s_max = t;
   L.i_max = t + (t + kItemRows - 1) / kItemRows;
   L.j_max = (3 * t + kMmaRows - 1) / kMmaRows + 1;
@@ -146,36 +182,66 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
+// Test a phase of an mbarrier; while it is incomplete the thread is
+// suspended in hardware (it issues nothing) until the phase completes or
+// about kSuspendNs pass.  Waiting warps thus leave the SM's issue slots to
+// the warps that have work.
+constexpr uint32_t kSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Wait for an mbarrier phase with an iteration cap and a 1 s wall-clock cap.
-// On giving up, records LORA_ERR_TIMEOUT in the sticky status and returns
-// false; the caller skips the work that needed the data.
+// Wait for an mbarrier phase with an iteration cap and a time cap (limit_ns,
+// 1 s unless the library's wait limit was lowered).  The time is counted in
+// SM clock cycles (clock64, a register read: the global timer costs far more
+// per read), two per nanosecond, which is at least limit_ns at any SM clock
+// up to 2 GHz.  On giving up, records LORA_ERR_TIMEOUT in the sticky status
+// and returns false; the caller skips the work that needed the data.
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr uint64_t kSpinNs = 1000000000ull;
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int *status) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int *status,
+                                                  uint64_t limit_ns = kSpinNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = global_timer_ns();
+  const long long t0 = clock64(), lim = (long long)(2 * limit_ns);
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 255u && global_timer_ns() - t0 > kSpinNs) break;
+    if (clock64() - t0 > lim) break;
+  }
+  atomicCAS(status, 0, LORA_ERR_TIMEOUT);
+  return false;
+}
+
+// Global-memory counters shared by the CTAs of one launch: an add with
+// release semantics (the adder's earlier writes become visible first) and a
+// load with acquire semantics, both at GPU scope.
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *p == want, bounded like mbar_wait_bounded.
+__device__ __forceinline__ bool wait_count_bounded(const unsigned *p, unsigned want, int *status,
+                                                   uint64_t limit_ns = kSpinNs) {
+  if (ld_acquire(p) == want) return true;
+  const long long t0 = clock64(), lim = (long long)(2 * limit_ns);
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    __nanosleep(64);  // (a poll is a global round trip; the sleep keeps the warp off the issue slots)
+    if (ld_acquire(p) == want) return true;
+    if (clock64() - t0 > lim) break;
   }
   atomicCAS(status, 0, LORA_ERR_TIMEOUT);
   return false;
@@ -267,9 +333,8 @@ struct lora_pool {
   void *dev_tables = nullptr;
   int32_t *d_pt = nullptr, *d_rank = nullptr, *d_loaded = nullptr;
   int *d_status = nullptr;
-  int decode_smem = 0;
-  int decode_max_clusters = 0;   // co-resident 8-CTA decode clusters
-  int decode_max_clusters4 = 0;  // co-resident 4-CTA decode clusters
+  int decode_per_sm = 0;    // co-resident decode CTAs per SM at this pool's r_max
+  int decode_max_ctas = 0;  // and on the whole device
   // Kind of the plan last built into each workspace (1 = index vector,
   // 2 = segments, which may hold tensor-core tiles); kept on the host so that
   // an apply call can pick its kernels without reading the device.
@@ -313,29 +378,37 @@ int launch_plan_ids(lora_pool *pool, const int32_t *ids, int T, void *ws, cudaSt
 int launch_plan_segments(lora_pool *pool, const int32_t *off, const int32_t *slot, int S, int T,
                          void *ws, cudaStream_t st);
 enum DecodeMode { kFused = 0, kShrinkOnly = 1, kExpandOnly = 2 };
-int launch_decode(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
-                  const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st);
-int launch_decode_items(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
-                        const float *scales, float *v, int ldv, int T, const void *ws, cudaStream_t st,
-                        int items_hdr);
-// Decode launch that groups ids[0 .. T) itself (T <= kFusedMaxT): no plan
-// kernel and no workspace.
-int launch_decode_ids(lora_pool *pool, int mode, int target, const void *x, int ldx, void *y, int ldy,
-                      const float *scales, float *v, int ldv, const int32_t *ids, int T, cudaStream_t st);
-// Fused decode over n_tgt targets that share x (same d_in and d_out); target
-// i writes columns y_cols[i] .. + d_out - 1 of y.  ids != nullptr: grouped in
-// the kernel (T <= kFusedMaxT); else the plan in ws.
-int launch_decode_multi(lora_pool *pool, int n_tgt, const int *targets, const int *y_cols, const void *x, int ldx,
-                        void *y, int ldy, const float *scales, const int32_t *ids, int T, const void *ws,
-                        cudaStream_t st);
-// Delta of routed expert pairs (pair p = token p / top_k, its (p % top_k)-th
-// expert; slot = adapter * n_experts + expert; x row p / top_k, y row p).
-// ws == nullptr: grouped in the kernel (n_pairs <= kFusedMaxT); else the plan
-// of the pairs' slots in ws.
-int launch_decode_moe(lora_pool *pool, int target, const void *x, int ldx, void *y, int ldy, const float *scales,
-                      const int32_t *lora_ids, const int32_t *topk, int n_pairs, int top_k, int n_experts,
-                      const void *ws, cudaStream_t st);
-// Writes each routed pair's slot (as launch_decode_moe forms it) to pair_ids.
+// One decode launch (decode.cu).  ids != nullptr: the kernel groups ids[0 ..
+// T) itself (T <= kFusedMaxT); else it reads the plan in ws (items counted by
+// header word items_hdr).  Targets share x,
+// d_in and d_out; target i writes columns y_cols[i] .. + d_out - 1 of y.
+// Routed expert pairs: x_div = top_k (row p reads x row p / top_k) and, for
+// in-kernel grouping, moe_topk / moe_k / moe_e form the pairs' slots.
+struct DecodeCall {
+  int mode = kFused;
+  int n_tgt = 1;
+  const int *targets = nullptr;
+  const int *y_cols = nullptr;
+  const void *x = nullptr;
+  int ldx = 0;
+  void *y = nullptr;
+  int ldy = 0;
+  const float *scales = nullptr;
+  float *v = nullptr;  // shrink-only output / expand-only input, [T, ldv] fp32
+  int ldv = 0;
+  int T = 0;
+  void *ws = nullptr;  // the plan (plan path only)
+  const int32_t *ids = nullptr;
+  int items_hdr = kHdrItems;
+  int x_div = 1;
+  const int32_t *moe_topk = nullptr;
+  int moe_k = 0, moe_e = 0;
+};
+int launch_decode(lora_pool *pool, const DecodeCall &c, cudaStream_t st);
+// Lowers (ns > 0) or restores (0) the wall-clock limit of the decode
+// kernel's bounded waits; 1 s by default.
+void set_wait_limit_ns(unsigned long long ns);
+// Writes each routed pair's slot (as the in-kernel grouping forms it) to pair_ids.
 int launch_moe_pair_ids(const lora_pool *pool, const int32_t *lora_ids, const int32_t *topk, int n_pairs,
                         int top_k, int n_experts, int32_t *pair_ids, cudaStream_t st);
 struct PrefillGeometry {

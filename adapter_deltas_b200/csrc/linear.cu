@@ -88,8 +88,7 @@ struct LnSmem {
   int *list;            // [256] slot of each adapter of the tile, by first row
   int *lrank;           // [256] its rank on the target
   float *lscale;        // [256] its scale
-  int *lpage;           // [256] physical page of its B^T row 0 in this tile (-1: none)
-  const uint8_t **brow; // [n_slots_d x 16] B^T row slices of the group's chunks (nullptr: crosses a page)
+  int *lpage;           // [256] physical page of its whole B^T block (-1: the block spans pages)
   int *gch;             // [n_slots_d] the group's chunks: adapter index << 8 | first rank row
   float *vst;           // [nt][v_cols] v of the tile's rows
   uint32_t *ballot;     // [8] first-row flags
@@ -107,7 +106,7 @@ __host__ __device__ inline int ln_ring_bytes(int nt, int ns) {
 }
 __host__ __device__ inline int ln_chunk_bytes(int nt) { return kLnBtBytes + ln_vv_bytes(nt); }
 __host__ __device__ inline int ln_fixed_bytes(int nd) {
-  return 1024 /* alignment slack */ + 6 * kLnMaxNT * 4 + nd * kLnChunk * 8 + ((nd * 4 + 15) & ~15) + 8 * 4 + 4 * 4 +
+  return 1024 /* alignment slack */ + 6 * kLnMaxNT * 4 + ((nd * 4 + 15) & ~15) + 8 * 4 + 4 * 4 +
          (2 * kLnMaxStages + 6) * 8 + 16;
 }
 __host__ __device__ inline int ln_vst_bytes(int nt, int v_cols) { return (nt * v_cols * 4 + 15) & ~15; }
@@ -138,19 +137,6 @@ __device__ __forceinline__ uint32_t ln_mapa(uint32_t addr, uint32_t cta) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(cta));
   return r;
 }
-// Page index of logical byte `off` of a slot, the offset inside that page
-// and the bytes left on it (the arithmetic of pool_addr without the lookup).
-__device__ __forceinline__ long long ln_page_of(const PoolView &p, long long off, long long *inside,
-                                                long long *room) {
-  if (p.log2_page < 0) {
-    *inside = off;
-    *room = p.page_bytes - off;
-    return 0;
-  }
-  *inside = off & (p.page_bytes - 1);
-  *room = p.page_bytes - *inside;
-  return off >> p.log2_page;
-}
 __device__ __forceinline__ void builders_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kLnBuilders) : "memory"); }
 
 __global__ void __launch_bounds__(kLnThreads, 1) linear_kernel(const __grid_constant__ LinearArgs a) {
@@ -176,7 +162,6 @@ __global__ void __launch_bounds__(kLnThreads, 1) linear_kernel(const __grid_cons
     S.bt = p; p += a.n_slots_d * kLnBtBytes;
     S.vv = p; p += a.n_slots_d * vv_bytes;
     S.vst = reinterpret_cast<float *>(p); p += ln_vst_bytes(NT, a.v_cols);
-    S.brow = reinterpret_cast<const uint8_t **>(p); p += a.n_slots_d * kLnChunk * 8;
     S.row_slot = reinterpret_cast<int *>(p); p += kLnMaxNT * 4;
     S.tok = reinterpret_cast<int *>(p); p += kLnMaxNT * 4;
     S.list = reinterpret_cast<int *>(p); p += kLnMaxNT * 4;
@@ -203,8 +188,6 @@ __global__ void __launch_bounds__(kLnThreads, 1) linear_kernel(const __grid_cons
   constexpr int kRowsPer = kLnMaxNT / kLnBuilders;
   int r_slot[kRowsPer], r_rank[kRowsPer], r_page[kRowsPer];
   float r_scale[kRowsPer];
-  long long in0, room0;
-  const long long page0 = ln_page_of(a.pool, a.bt_off + (long long)m0 * 2, &in0, &room0);
   if (warp < 4) {
     int id[kRowsPer];
 #pragma unroll
@@ -218,7 +201,7 @@ __global__ void __launch_bounds__(kLnThreads, 1) linear_kernel(const __grid_cons
       const int ld = in ? a.pool.loaded[id[q]] : 0;
       const int r = in ? a.pool.rank[id[q] * a.pool.n_targets + a.target] : 0;
       r_scale[q] = in ? a.scales[id[q]] : 0.f;
-      r_page[q] = in ? a.pool.pt[(long long)id[q] * a.pool.pps + page0] : -1;
+      r_page[q] = in ? block_page(a.pool, id[q], a.bt_off, (long long)a.pool_r_max * a.d_out * 2) : -1;
       const bool ok = ld && r > 0 && r <= a.pool_r_max;
       r_slot[q] = ok ? id[q] : -1;
       r_rank[q] = ok ? r : 0;
@@ -385,24 +368,6 @@ __global__ void __launch_bounds__(kLnThreads, 1) linear_kernel(const __grid_cons
       }
       builders_sync();
       const int n_in = min(ND, nch - g * ND);
-      const int cols = min(kMmaRows, a.d_out - m0);
-      for (int e = tid; e < n_in * kLnChunk; e += kLnBuilders) {
-        const int ch = S.gch[e / kLnChunk];
-        const int j = (ch & 255) + e % kLnChunk;
-        const uint8_t *p = nullptr;
-        if (j < a.pool_r_max) {
-          const int ai = ch >> 8;
-          const long long off = a.bt_off + ((long long)j * a.d_out + m0) * 2;
-          long long inside, room;
-          if (ln_page_of(a.pool, off, &inside, &room) == page0 && S.lpage[ai] >= 0)
-            p = a.pool.base + (long long)S.lpage[ai] * a.pool.page_bytes + inside;  // the page of row 0
-          else
-            p = pool_addr(a.pool, S.list[ai], off, &room);
-          if (p && room < (long long)cols * 2) p = nullptr;
-        }
-        S.brow[e] = p;
-      }
-      builders_sync();
       return n_in;
     };
     // B^T rows j0 .. j0 + 15 of the tile's 128 features, feature-major core
@@ -418,12 +383,13 @@ __global__ void __launch_bounds__(kLnThreads, 1) linear_kernel(const __grid_cons
         const uint32_t dst = bt_u + b * kLnBtBytes + jg * kLnBtLbo + nv * 128 + jl * 16;
         const uint8_t *src = nullptr;
         if (j < a.pool_r_max && f < a.d_out) {
-          src = S.brow[b * kLnChunk + row];
-          if (src) {
-            src += nv * 16;
-          } else {  // the slice crosses a page: look this 16-byte piece up
+          const long long off = a.bt_off + block_chunk_off(j, f / 8, a.d_out, a.pool_r_max);
+          const int pg = S.lpage[ch >> 8];
+          if (pg >= 0) {
+            src = page_addr(a.pool, pg, off);
+          } else {  // the block spans pages: look this 16-byte piece up
             long long room;
-            src = pool_addr(a.pool, S.list[ch >> 8], a.bt_off + ((long long)j * a.d_out + f) * 2, &room);
+            src = pool_addr(a.pool, S.list[ch >> 8], off, &room);
           }
         }
         if (src)

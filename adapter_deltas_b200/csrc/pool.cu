@@ -69,20 +69,24 @@ static void for_each_run(const lora_pool *p, int slot, long long off, long long 
   }
 }
 
-// B (d_out x rank, row-major) -> rows j of B^T in the pool, through the page
-// table.  One thread per 8 consecutive output columns of one row j.
-__global__ void store_bt_kernel(PoolView pool, int slot, long long bt_off, int d_out, int rank,
-                                const uint16_t *B) {
-  long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  long long per_row = d_out / 8;
-  if (idx >= per_row * rank) return;
-  int j = (int)(idx / per_row);
-  int n0 = (int)(idx % per_row) * 8;
-  uint16_t v[8];
+// One block of a slot written whole, in the pool's tiled arrangement
+// (block_chunk_off): rows below `rank` from src, the rank padding as zeros.
+// src is A (rank x width, row-major; transposed = 0) or B (width x rank,
+// row-major; transposed = 1, stored as B^T).  One thread per 16-byte chunk.
+__global__ void store_block_kernel(PoolView pool, int slot, long long blk_off, int width, int r_max, int rank,
+                                   const uint16_t *src, int transposed) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nch = width / 8;
+  if (idx >= (long long)nch * r_max) return;
+  const int j = (int)(idx / nch), c = (int)(idx % nch);
+  uint16_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (j < rank) {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) v[e] = B[(long long)(n0 + e) * rank + j];
+    for (int e = 0; e < 8; ++e)
+      v[e] = transposed ? src[(long long)(c * 8 + e) * rank + j] : src[(long long)j * width + c * 8 + e];
+  }
   long long room;
-  const uint8_t *dst = pool_addr(pool, slot, bt_off + ((long long)j * d_out + n0) * 2, &room);
+  const uint8_t *dst = pool_addr(pool, slot, blk_off + block_chunk_off(j, c, width, r_max), &room);
   if (!dst) return;
   uint4 packed;
   packed.x = v[0] | (uint32_t(v[1]) << 16);
@@ -90,6 +94,19 @@ __global__ void store_bt_kernel(PoolView pool, int slot, long long bt_off, int d
   packed.z = v[4] | (uint32_t(v[5]) << 16);
   packed.w = v[6] | (uint32_t(v[7]) << 16);
   *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(dst)) = packed;
+}
+
+// Host image of one block in the tiled arrangement (see store_block_kernel).
+static void block_image(const uint16_t *src, int transposed, int width, int r_max, int rank,
+                        std::vector<uint16_t> *img) {
+  img->assign((size_t)r_max * width, 0);
+  const int nch = width / 8;
+  for (int j = 0; j < rank; ++j)
+    for (int c = 0; c < nch; ++c) {
+      uint16_t *d = img->data() + block_chunk_off(j, c, width, r_max) / 2;
+      for (int e = 0; e < 8; ++e)
+        d[e] = transposed ? src[(size_t)(c * 8 + e) * rank + j] : src[(size_t)j * width + c * 8 + e];
+    }
 }
 
 // One target's part of a swap-in: where its A (then its B) sits in the
@@ -115,12 +132,12 @@ __global__ void swap_in_kernel(PoolView pool, int slot, int r_max, const SwapDes
     long long off;
     if (c < na) {
       const int j = (int)(c / per_a);
-      off = d.a_off + c * 16;
+      off = d.a_off + block_chunk_off(j, (int)(c % per_a), d.d_in, r_max);
       if (j < d.rank) v = *reinterpret_cast<const uint4 *>(data + d.src + c * 16);
     } else {
       const long long cb = c - na;
       const int j = (int)(cb / per_b), n0 = (int)(cb % per_b) * 8;
-      off = d.bt_off + cb * 16;
+      off = d.bt_off + block_chunk_off(j, (int)(cb % per_b), d.d_out, r_max);
       if (j < d.rank) {
         uint16_t e[8];
 #pragma unroll
@@ -302,37 +319,35 @@ int lora_pool_load(lora_pool *p, int slot, int target, int rank, const void *A, 
   }
 
   const long long a_off = p->a_off[target], bt_off = p->bt_off[target];
-  const long long a_used = (long long)rank * d_in * 2, a_all = (long long)p->r_max * d_in * 2;
-  const long long b_used = (long long)rank * d_out * 2, b_all = (long long)p->r_max * d_out * 2;
-  const cudaMemcpyKind kind = src_is_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  const long long a_all = (long long)p->r_max * d_in * 2, b_all = (long long)p->r_max * d_out * 2;
   int rc = LORA_OK;
-  auto copy = [&](const uint8_t *src) {
-    return [&, src](uint8_t *dst, long long done, long long n) {
-      if (rc == LORA_OK && cudaMemcpyAsync(dst, src + done, (size_t)n, kind, st) != cudaSuccess) rc = LORA_ERR_CUDA;
+  if (src_is_device) {
+    // one kernel per block: the rows in the pool's tiled arrangement, B
+    // transposed, the rank padding zeroed
+    const int threads = 256;
+    const long long na = (long long)p->r_max * (d_in / 8), nb = (long long)p->r_max * (d_out / 8);
+    g_launches.fetch_add(2);
+    store_block_kernel<<<(unsigned)((na + threads - 1) / threads), threads, 0, st>>>(
+        p->view(), slot, a_off, d_in, p->r_max, rank, static_cast<const uint16_t *>(A), 0);
+    store_block_kernel<<<(unsigned)((nb + threads - 1) / threads), threads, 0, st>>>(
+        p->view(), slot, bt_off, d_out, p->r_max, rank, static_cast<const uint16_t *>(B), 1);
+    if (cudaGetLastError() != cudaSuccess) rc = LORA_ERR_CUDA;
+  } else {
+    // host images of both blocks, each copied as one logical range (cut at
+    // page boundaries)
+    std::vector<uint16_t> ia, ib;
+    block_image(static_cast<const uint16_t *>(A), 0, d_in, p->r_max, rank, &ia);
+    block_image(static_cast<const uint16_t *>(B), 1, d_out, p->r_max, rank, &ib);
+    auto copy = [&](const uint8_t *src) {
+      return [&, src](uint8_t *dst, long long done, long long n) {
+        if (rc == LORA_OK && cudaMemcpyAsync(dst, src + done, (size_t)n, cudaMemcpyHostToDevice, st) != cudaSuccess)
+          rc = LORA_ERR_CUDA;
+      };
     };
-  };
-  auto zero = [&](uint8_t *dst, long long, long long n) {
-    if (rc == LORA_OK && cudaMemsetAsync(dst, 0, (size_t)n, st) != cudaSuccess) rc = LORA_ERR_CUDA;
-  };
-  if (rank > 0) {
-    for_each_run(p, slot, a_off, a_used, copy(static_cast<const uint8_t *>(A)));
-    if (src_is_device) {
-      long long n = (long long)rank * (d_out / 8);
-      int threads = 256;
-      g_launches.fetch_add(1);
-      store_bt_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
-          p->view(), slot, bt_off, d_out, rank, static_cast<const uint16_t *>(B));
-      if (cudaGetLastError() != cudaSuccess) rc = LORA_ERR_CUDA;
-    } else {
-      const uint16_t *Bh = static_cast<const uint16_t *>(B);
-      std::vector<uint16_t> bt((size_t)rank * d_out);
-      for (int n = 0; n < d_out; ++n)
-        for (int j = 0; j < rank; ++j) bt[(size_t)j * d_out + n] = Bh[(size_t)n * rank + j];
-      for_each_run(p, slot, bt_off, b_used, copy(reinterpret_cast<const uint8_t *>(bt.data())));
-    }
+    for_each_run(p, slot, a_off, a_all, copy(reinterpret_cast<const uint8_t *>(ia.data())));
+    for_each_run(p, slot, bt_off, b_all, copy(reinterpret_cast<const uint8_t *>(ib.data())));
+    if (rc == LORA_OK && cudaStreamSynchronize(st) != cudaSuccess) rc = LORA_ERR_CUDA;  // the images go out of scope
   }
-  if (a_all > a_used) for_each_run(p, slot, a_off + a_used, a_all - a_used, zero);
-  if (b_all > b_used) for_each_run(p, slot, bt_off + b_used, b_all - b_used, zero);
   if (rc != LORA_OK) {
     (void)cudaGetLastError();
     return rc;
@@ -341,7 +356,6 @@ int lora_pool_load(lora_pool *p, int slot, int target, int rank, const void *A, 
   CUDA_TRY(cudaMemcpyAsync(p->d_rank + (size_t)slot * p->n_targets + target,
                            p->rank.data() + (size_t)slot * p->n_targets + target, 4,
                            cudaMemcpyHostToDevice, st));
-  if (!src_is_device) CUDA_TRY(cudaStreamSynchronize(st));  // host staging buffers go out of scope
   return LORA_OK;
 }
 
@@ -459,7 +473,7 @@ int lora_pool_get_info(const lora_pool *p, lora_pool_info *info) {
   info->n_slots = p->n_slots;
   info->n_targets = p->n_targets;
   info->r_max = p->r_max;
-  info->decode_clusters = p->decode_max_clusters;
+  info->decode_ctas = p->decode_max_ctas;
   return LORA_OK;
 }
 

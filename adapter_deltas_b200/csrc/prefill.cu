@@ -80,13 +80,13 @@ struct __align__(64) PrefillArgs {
   int n_groups;         // expand column groups
 };
 
-// Address of 16-byte chunk `chunk` of a rank row slice: from the row's start
-// when the slice lies on one page, else through the page table.
-__device__ __forceinline__ const uint8_t *slice_chunk(const PoolView &pool, int slot, const uint8_t *row_start,
-                                                      long long row_off, int chunk, int *status) {
-  if (row_start) return row_start + chunk * 16;
+// Address of the 16-byte chunk at logical byte `off` of a slot's block: on
+// the block's page when it has one (page >= 0), else through the page table.
+__device__ __forceinline__ const uint8_t *block_chunk(const PoolView &pool, int slot, int page, long long off,
+                                                      int *status) {
+  if (page >= 0) return page_addr(pool, page, off);
   long long room;
-  const uint8_t *src = pool_addr(pool, slot, row_off + (long long)chunk * 16, &room);
+  const uint8_t *src = pool_addr(pool, slot, off, &room);
   if (!src) {
     set_status(status, LORA_ERR_NOT_LOADED);
     src = pool.base;
@@ -188,16 +188,22 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     // The A slice does not wait for the rank: all r_cap rows come (the pool
     // keeps an adapter's rows past its rank at zero), so the copies leave as
     // soon as the tile record is known.
+    // The slice is whole pool tiles (k-slices start on tile boundaries): the
+    // first rows_cp rows of each tile are one contiguous range of the block,
+    // copied as they are (tile after tile, tile stride r_cap rows).
     const int cols = min(nkb * kBoxCols, a.d_in - kb0 * kBoxCols);
-    const uint32_t row_bytes = (uint32_t)cols * 2u, stg_pitch = (uint32_t)a.kb_per * kBoxCols * 2u;
-    const long long row_off0 = a.a_off + (long long)kb0 * kBoxCols * 2;
+    const int tc = pool_tile_cols(a.pool_r_max), tcc = tc / 8;
+    const int tile0 = kb0 * kBoxCols / tc, n_tl = (cols + tc - 1) / tc;
     const int rows_cp = min(a.r_cap, a.pool_r_max);
     if (warp == 0) {
-      if (lane == 0) mbar_arrive_expect_tx(S.a_land, (uint32_t)rows_cp * row_bytes);
+      if (lane == 0) mbar_arrive_expect_tx(S.a_land, (uint32_t)rows_cp * (uint32_t)cols * 2u);
       __syncwarp();
-      if (lane < rows_cp)
-        copy_pool_row(a.pool, slot, row_off0 + (long long)lane * a.d_in * 2, row_bytes, S.stg + lane * stg_pitch,
-                      S.a_land, a.status);
+      if (lane < n_tl) {
+        const int t = tile0 + lane;
+        const int tw = min(tcc, a.d_in / 8 - t * tcc);
+        copy_pool_row(a.pool, slot, a.a_off + (long long)t * a.pool_r_max * tcc * 16, (uint32_t)(rows_cp * tw * 16),
+                      S.stg + lane * a.r_cap * tcc * 16, S.a_land, a.status);
+      }
     }
     const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
     const bool use = r > 0 && r <= a.r_cap;
@@ -229,11 +235,11 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
       __syncwarp();
     } else {
       // ------------------------------------------------ epilogue warps
-      // (1) the k-slice of A_a, copied above into a row-major staging area
-      // (one bulk copy per row, pieces where a row crosses a page), moved
-      // into the MMA's K-major core-matrix layout: 8 rank rows x 4 chunks per
-      // warp access, so each 128-byte core matrix is written whole; zero rows
-      // from r up to R and zero columns beyond d_in
+      // (1) the k-slice of A_a, copied above in the pool's tiled arrangement
+      // (one bulk copy per tile), moved into the MMA's K-major core-matrix
+      // layout: 8 rank rows x 4 chunks per warp access, so each 128-byte core
+      // matrix is written whole; zero rows from r up to R and zero columns
+      // beyond d_in
       warp_wait(S.a_land, ucopy & 1u, a.status, alive);
       if (use) {
         const int kv_n = nkb * (kBoxCols / 8);
@@ -242,7 +248,11 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
           const int j = jg * 8 + jl;
           for (int kv = warp * 4 + vo; kv < kv_n; kv += kShEpiWarps * 4) {
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (j < r && kv * 8 < cols) v = *reinterpret_cast<const uint4 *>(S.stg + j * stg_pitch + kv * 16);
+            if (j < r && kv * 8 < cols) {
+              const int tl = kv / tcc, c = kv - tl * tcc;
+              const int tw = min(tcc, a.d_in / 8 - (tile0 + tl) * tcc);
+              v = *reinterpret_cast<const uint4 *>(S.stg + (tl * a.r_cap * tcc + j * tw + swz_chunk(c, j, tw)) * 16);
+            }
             *reinterpret_cast<uint4 *>(S.aw + kv * lbo_a + jg * 128 + jl * 16) = v;
           }
         }
@@ -288,14 +298,13 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
 // ============================================================ expand kernel
 struct ExSmem {
   uint8_t *ys, *bw, *vop;
-  const uint8_t **brow;
   uint64_t *y_full, *mma_done;
   uint32_t *tmem_slot;
 };
 
 __host__ __device__ inline int ex_smem_bytes(int r_cap) {
   return 1024 /* alignment slack */ + kGroupBoxes * kBoxBytes + r_cap * kGroupCols * 2 + 2 * kMmaRows * r_cap * 2 +
-         kPfRankCap * 8 + 2 * 8 + 16;
+         2 * 8 + 16;
 }
 
 // Every warp takes every step of a unit; several CTAs per SM overlap one's
@@ -311,7 +320,6 @@ __global__ void __launch_bounds__(kExThreads, kExMaxPerSm) pf_expand_kernel(cons
     S.ys = p; p += kGroupBoxes * kBoxBytes;
     S.bw = p; p += a.r_cap * kGroupCols * 2;
     S.vop = p; p += 2 * kMmaRows * a.r_cap * 2;
-    S.brow = reinterpret_cast<const uint8_t **>(p); p += kPfRankCap * 8;
     uint64_t *b = reinterpret_cast<uint64_t *>(p);
     S.y_full = b++;
     S.mma_done = b++;
@@ -364,19 +372,16 @@ __global__ void __launch_bounds__(kExThreads, kExMaxPerSm) pf_expand_kernel(cons
     }
     // (2) B^T columns of the unit (rows < r; zero rows up to R and columns
     // beyond d_out) in the MMA's MN-major core-matrix layout
-    const long long row_off0 = a.bt_off + (long long)col_base * 2;
-    if (tid < r) {
-      long long room;
-      const uint8_t *p = pool_addr(a.pool, slot, row_off0 + (long long)tid * a.d_out * 2, &room);
-      S.brow[tid] = (p && room >= (long long)cols * 2) ? p : nullptr;
-    }
-    __syncthreads();
+    // (chunks located through the pool's tiled arrangement of the block)
+    const int bpage = block_page(a.pool, slot, a.bt_off, (long long)a.pool_r_max * a.d_out * 2);
     for (int idx = tid; idx < R * (kGroupCols / 8); idx += kExThreads) {
       const int jl = idx & 7, nv = (idx >> 3) & (kGroupCols / 8 - 1), jg = idx / (8 * (kGroupCols / 8));
       const int j = jg * 8 + jl;
       const uint32_t dst = bw_u + jg * lbo_b + nv * 128 + jl * 16;
       if (j < r && nv * 8 < cols)
-        cp_async16_pf(dst, slice_chunk(a.pool, slot, S.brow[j], row_off0 + (long long)j * a.d_out * 2, nv, a.status));
+        cp_async16_pf(dst, block_chunk(a.pool, slot, bpage,
+                                       a.bt_off + block_chunk_off(j, col_base / 8 + nv, a.d_out, a.pool_r_max),
+                                       a.status));
       else
         st_shared_zero16(dst);
     }
@@ -518,8 +523,11 @@ bool prefill_geometry(const lora_pool *pool, int target, int max_tiles, PrefillG
   const int r_cap = pool->r_max <= 16 ? 16 : 32;
   const int nkb_all = (d_in + kBoxCols - 1) / kBoxCols;
   const int want_ks = std::max(1, (kSms + std::max(max_tiles, 1) - 1) / std::max(max_tiles, 1));
+  // k-slices of whole pool tiles (the shrink copies its adapter slice one
+  // tile at a time)
+  const int tb = pool_tile_cols(pool->r_max) / kBoxCols;
   int kb_per = (nkb_all + want_ks - 1) / want_ks;
-  kb_per = std::max(4, std::min(kShMaxBlocks, kb_per));
+  kb_per = std::max(tb, std::min(kShMaxBlocks, (kb_per + tb - 1) / tb * tb));
   kb_per = std::min(kb_per, nkb_all);
   const int cap = 227 * 1024;
   int ns = 0;

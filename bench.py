@@ -87,7 +87,10 @@ def traffic_from_profile(kernel: str, kernel_file: str, workload: str):
         if ":" in ln:
             k, v = ln.split(":", 1)
             kv[k.strip()] = v.strip()
-    src = open(os.path.join(ROOT, "adapter_deltas_b200", "csrc", kernel_file), "rb").read()
+    try:
+        src = open(os.path.join(ROOT, "adapter_deltas_b200", "csrc", kernel_file), "rb").read()
+    except OSError:
+        return None
     if kv.get("source_sha256") != hashlib.sha256(src).hexdigest():
         return None
     try:
@@ -447,7 +450,7 @@ def run_b200(args, rank: int, world: int, local_rank: int):
         "hbm_gbs_step": alg * world / (ms * 1e-3) / 1e9 / world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": traffic_from_profile(kernel_name, "prefill.cu" if segmented else "sgmv.cu",
+                     "traffic": traffic_from_profile(kernel_name, "prefill.cu" if segmented else "decode.cu",
                                                      args.workload),
                      "traffic_note": "DRAM bytes of one launch (prefill: shrink + expand launches) from the ncu "
                                      "summary in profiles/, while its source hash matches",
@@ -580,7 +583,7 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
                    "deltas_per_step": n_t, "l2": "pool 31.25 GiB and 1 GiB of activations per step > L2",
                    "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "sgmv.cu", "paged"),
+                     "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "decode.cu", "paged"),
                      "kernel": "decode_kernel<fused>", "kernel_us": kernel_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg},
         "e2e": {"value": job_value(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -967,7 +970,7 @@ def run_moe(args, rank, world, dev, bf16):
                    "l2": "%d rotating buffer sets, %.0f MB > 4x L2" % (n_sets, n_sets * set_bytes / 1e6),
                    "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "sgmv.cu", "moe"),
+                     "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "decode.cu", "moe"),
                      "traffic_note": "DRAM bytes of one launch from the ncu summary in profiles/, while its "
                                      "source hash matches",
                      "kernel": "decode_kernel<fused> forming and grouping the pairs' slots in-kernel (the whole step)",

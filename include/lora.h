@@ -95,6 +95,17 @@ typedef struct {
  * section "Where does multi-LoRA serving actually break?", item 2); kernels
  * read only the adapter's own rank.
  *
+ * Inside a block of `width` columns the rows are stored in column tiles of
+ * tc = 1024 columns (r_max <= 16), 512 (r_max <= 32) or 256 (r_max > 32),
+ * so that r_max rows of a tile are 32 KiB: tile k
+ * holds columns k*tc .. min((k+1)*tc, width)-1 of rows 0..r_max-1, row after
+ * row (tw = that tile's width in 16-byte chunks of 8 columns), and starts at
+ * byte k * r_max * tc * 2 of the block.  In a row of a tile, chunk c of every
+ * complete group of eight chunks is stored at position c ^ (row % 8); a
+ * trailing partial group keeps its order.  The first r rows of a tile are
+ * thus one contiguous range (the decode kernel stages them with one copy),
+ * and the rows of a staged tile fall in different shared-memory banks.
+ *
  * Paging.  A slot's logical bytes are cut into pages of page_bytes; page p of
  * slot s lives at physical page page_table[s * pages_per_slot + p], i.e. at
  * byte pool_mem + page * page_bytes.  page_bytes == 0 means one page per slot
@@ -194,8 +205,8 @@ typedef struct {
     int n_pages;            /* physical pages in pool_mem                    */
     int free_pages;
     int n_slots, n_targets, r_max;
-    int decode_clusters;    /* thread-block clusters of the decode kernel
-                               that can be resident at once on this device */
+    int decode_ctas;        /* CTAs of the decode kernel that can be
+                               resident at once on this device */
 } lora_pool_info;
 
 LORA_API int lora_pool_get_info(const lora_pool *pool, lora_pool_info *info);
@@ -212,7 +223,9 @@ LORA_API int lora_pool_target_offsets(const lora_pool *pool, int target,
  * tiles), then, where the tensor-core segment path can serve the target, the
  * fp32 partial V of each k-slice of d_in (T x slices x rank bound x 4 bytes).
  * A workspace shared by several targets takes the largest of their sizes.
- * Calls with a smaller workspace return LORA_ERR_WORKSPACE.
+ * Calls with a smaller workspace return LORA_ERR_WORKSPACE.  Its contents
+ * need no initialisation; calls that overlap on the GPU need workspaces of
+ * their own.
  */
 LORA_API size_t lora_workspace_bytes(const lora_pool *pool, int target, int max_tokens);
 
@@ -447,20 +460,23 @@ LORA_API int lora_expand(lora_pool *pool, int target, const float *v, int ldv, v
  * front), or they run in a loop that cannot afford the device-wide
  * synchronisation that cudaMalloc / cudaFree may cause.
  *
- * The call computes exactly what lora_apply computes, with the same
- * arguments minus ws / ws_bytes.  The plan lives in one fixed array of device
- * memory compiled into the library (138,800 bytes, enough for
- * LORA_NOALLOC_MAX_TOKENS rows); every GPU that loads the library holds that
- * array until the process exits.  The call itself allocates nothing.
+ * The call computes exactly what lora_apply computes (bit for bit), with the
+ * same arguments minus ws / ws_bytes.  Batches of at most 256 rows take one
+ * launch that needs no plan, as in lora_apply.  Larger batches keep their
+ * plan in one fixed array of device memory compiled into the library
+ * (137,472 bytes, enough for LORA_NOALLOC_MAX_TOKENS rows); every GPU that loads
+ * the library holds that array until the process exits.  The call itself
+ * allocates nothing.
  *   - T > LORA_NOALLOC_MAX_TOKENS returns LORA_ERR_WORKSPACE (nothing runs).
  *   - The first call on a device looks up the array's device address (a
- *     runtime query, done once per device with that device current); make
- *     that first call before capturing a stream into a CUDA graph.
- *   - All calls share the one array, which keeps the last call's plan.  No
- *     part of it needs clearing (each call rewrites everything it reads), but
- *     calls that overlap on the GPU -- on different streams, or on different
- *     pools of the same device -- race on it and must be serialised by the
- *     caller.
+ *     runtime query, done with that device current, and again after a device
+ *     reset or from another driver context); make that first call before
+ *     capturing a stream into a CUDA graph.
+ *   - All calls of more than 256 rows share the one array, which keeps the
+ *     last call's plan.  No part of it needs clearing (each call rewrites
+ *     everything it reads), but such calls that overlap on the GPU -- on
+ *     different streams, or on different pools of the same device -- race on
+ *     it and must be serialised by the caller.
  */
 LORA_API int lora_apply_noalloc(lora_pool *pool, int target, const void *x, int ldx, void *y,
                                 int ldy, const int32_t *ids, const float *scales, int T,
@@ -474,6 +490,16 @@ LORA_API int lora_get_error(lora_pool *pool, int *device_status, void *stream);
 
 /* Number of kernels this library has launched in this process. */
 LORA_API uint64_t lora_kernel_launches(void);
+
+/*
+ * Wall-clock limit of the decode kernel's bounded waits (for a stage of its
+ * copy ring, or for the shrink partials of an item), in nanoseconds, for the
+ * launches that follow; 0 restores the default of one second.  A wait that
+ * runs out sets LORA_ERR_TIMEOUT in the pool's sticky status, leaves the
+ * rows that needed the data untouched and lets the kernel finish; it never
+ * faults.  Tests lower it to reach that path quickly.
+ */
+LORA_API void lora_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

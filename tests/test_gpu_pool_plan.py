@@ -134,6 +134,28 @@ def _reconstruct(pool_mem, pt, slot, layout, pps, page_bytes, slot_bytes):
     return logical[:slot_bytes]
 
 
+def _untile(block: np.ndarray, r_max: int, width: int) -> np.ndarray:
+    """A block [r_max, width] (bf16 bits) from its stored arrangement, as the
+    header states it: column tiles of 1024 columns (r_max <= 16), 512 (r_max
+    <= 32) or 256, each
+    tile the rows one after the other, the 16-byte chunks of each complete
+    group of eight in a row stored at chunk ^ (row % 8)."""
+    tcc = (1024 if r_max <= 16 else 512 if r_max <= 32 else 256) // 8
+    nch = width // 8
+    u = block.view(np.uint16)
+    out = np.empty((r_max, width), np.uint16)
+    base = 0
+    for k in range(-(-nch // tcc)):
+        tw = min(tcc, nch - k * tcc)
+        tile = u[base:base + r_max * tw * 8].reshape(r_max, tw, 8)
+        c = np.arange(tw)[None, :]
+        j = np.arange(r_max)[:, None]
+        pos = np.where((c | 7) < tw, c ^ (j & 7), c)
+        out[:, k * tcc * 8:(k * tcc + tw) * 8] = tile[j, pos].reshape(r_max, tw * 8)
+        base += r_max * tcc * 8
+    return out
+
+
 @pytest.mark.parametrize("cfg,page", [(1, 4096), (4, 1 << 16), (2, 0)])
 def test_pool_reconstruction_bitwise(cuda_device, cfg, page):
     w = synth.config(cfg)
@@ -152,8 +174,8 @@ def test_pool_reconstruction_bitwise(cuda_device, cfg, page):
             for t, (d_in, d_out) in enumerate(w.targets):
                 A, B = w.adapter(s, t)
                 a0, b0 = int(layout[0][t]), int(layout[1][t])
-                Ap = logical[a0:a0 + w.r_max * d_in * 2].view(np.uint16).reshape(w.r_max, d_in)
-                Bt = logical[b0:b0 + w.r_max * d_out * 2].view(np.uint16).reshape(w.r_max, d_out)
+                Ap = _untile(logical[a0:a0 + w.r_max * d_in * 2], w.r_max, d_in)
+                Bt = _untile(logical[b0:b0 + w.r_max * d_out * 2], w.r_max, d_out)
                 assert np.array_equal(Ap[:r], A) and not Ap[r:].any()
                 assert np.array_equal(Bt[:r], B.T) and not Bt[r:].any()
 
