@@ -46,6 +46,9 @@ constexpr int kDecThreads = kDecWarps * 32;
 // whose ring fills one SM's shared memory (one CTA, registers to spare); the
 // other ranks' rings fit twice.
 constexpr int dec_min_blocks(int jb) { return jb == 2 ? 1 : 2; }
+// 16-byte chunks per row of a full pool tile for the kernel's rank class
+// (the tile width of the largest rank the class serves).
+__host__ __device__ constexpr int full_tile_chunks(int jb) { return pool_tile_cols(8 * jb) / 8; }
 constexpr int kCacheItems = 256;  // items whose records a CTA keeps in shared memory
 constexpr int kCachePerm = 512;   // grouped row positions a CTA keeps in shared memory
 
@@ -122,6 +125,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
+}
+__device__ __forceinline__ void stsm_x4(uint32_t addr, const uint32_t (&r)[4]) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
 }
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -225,6 +233,66 @@ __device__ __forceinline__ void shrink_mma(uint32_t buf_u, uint32_t act_u, int p
   }
 }
 
+// The same over a full tile (wv = the pool's tile width, every chunk in a
+// complete group of eight): the warp's KPW k-steps have compile-time
+// positions; their operands are loaded in batches of k-steps (four; two
+// for ranks past 16, one past 32) ahead of the MMAs, and consecutive k-steps alternate between two
+// accumulator sets (added at the end, in fixed order; ranks up to 32 --
+// beyond, the warp's two k-steps have eight chains already).
+template <int JB, int KPW>
+__device__ __forceinline__ void shrink_full(uint32_t buf_u, uint32_t act_u, int pitch, int wv, int r, int m,
+                                            float (&acc)[JB < 2 ? 2 : JB][4], int lane, int warp) {
+  constexpr int NT = JB < 2 ? 2 : JB;
+  constexpr int NP = NT / 2;
+  constexpr int BATCH = NP >= 4 ? 1 : NP >= 2 ? 2 : KPW < 4 ? KPW : 4;  // k-steps whose operands load together
+  const int xr = (lane & 7) + ((lane >> 3) & 1) * 8, xk = (lane >> 4) * 16;
+  const uint32_t xrow = act_u + (xr < m ? xr : 0) * pitch + xk;
+  const int ahalf = (lane >> 3) & 1;
+  uint32_t abase[NP], ax[NP];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int j = (lane & 7) + (lane >> 4) * 8 + 16 * p;
+    const int jr = j < r ? j : 0;
+    abase[p] = buf_u + (uint32_t)(jr * wv) * 16u;
+    ax[p] = (uint32_t)(jr & 7);
+  }
+  const int np = min(NP, (r + 15) >> 4);
+  float acc2[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc2[nt][0] = acc2[nt][1] = acc2[nt][2] = acc2[nt][3] = 0.f;
+#pragma unroll
+  for (int b0 = 0; b0 < KPW; b0 += BATCH) {
+    uint32_t xa[BATCH][4], wa[BATCH][NP][4];
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) ldsm_x4(xrow + (warp + kConsumerWarps * (b0 + i)) * 32, xa[i]);
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const uint32_t c = (uint32_t)(2 * (warp + kConsumerWarps * (b0 + i)) + ahalf);
+#pragma unroll
+      for (int p = 0; p < NP; ++p)
+        if (p < np) ldsm_x4(abase[p] + ((c ^ ax[p]) << 4), wa[i][p]);
+    }
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      float(&dst)[NT][4] = (NT <= 4 && ((b0 + i) & 1)) ? acc2 : acc;
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        if (p < np) {
+          mma_bf16_16816(dst[2 * p], xa[i], wa[i][p][0], wa[i][p][1]);
+          mma_bf16_16816(dst[2 * p + 1], xa[i], wa[i][p][2], wa[i][p][3]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    acc[nt][0] += acc2[nt][0];
+    acc[nt][1] += acc2[nt][1];
+    acc[nt][2] += acc2[nt][2];
+    acc[nt][3] += acc2[nt][3];
+  }
+}
+
 // This warp's partial V of the item -> red[i * r + j] (rows < m, ranks < r).
 template <int JB>
 __device__ __forceinline__ void shrink_spill(const float (&acc)[JB < 2 ? 2 : JB][4], int r, int m, float *red,
@@ -269,49 +337,85 @@ __device__ __forceinline__ void expand_prepare(const float *s_v, int ld, int r, 
   }
 }
 
-// G column groups of this warp at once (cg0, cg0 + gstep, ...; ng <= G of
-// them), so that the MMA chains of the groups overlap.  Each group's
-// accumulator takes, per 16-rank block, the hi term and then the lo term.
-template <int JB, int G>
-__device__ __forceinline__ void expand_groups(uint32_t buf_u, const uint8_t *yb, uint32_t zero_u, int pitch, int wv,
-                                              int v_lo, int r, int m, const ExpandA<JB> &A, float scale,
-                                              const int *s_rows, long long ycol, const DecodeArgs &a, int lane,
-                                              int cg0, int gstep, int ng) {
+// Per-lane addressing of one expand tile, set up once per tile.  Lane
+// (g = lane / 4, t = lane % 4) owns output rows g and g + 8 and, in every
+// 8-column n-tile, columns 2t and 2t + 1; its ldmatrix row is rank
+// 16 ks + bj of chunk half bc.
+struct ExpandLane {
+  uint32_t rb[4];        // per 16-rank block: the lane's B^T row (or 16 zero bytes past the rank)
+  uint32_t xm[4], cm[4]; // its swizzle (row % 8) and chunk mask (0 for the zero row)
+  uint8_t *ys0, *ys1;    // staged y of rows g, g + 8 at column 2t (updated in place)
+  bool ok0, ok1;         // rows g, g + 8 belong to the item
+  int bc, nks;
+};
+
+template <int JB>
+__device__ __forceinline__ ExpandLane expand_lane(uint32_t buf_u, uint8_t *yb, uint32_t zero_u, int pitch, int wv,
+                                                  int r, int m, int lane) {
+  ExpandLane L;
   const int g = lane >> 2, t = lane & 3;
-  const int bj = (lane & 7) + ((lane >> 3) & 1) * 8, bc = lane >> 4;
+  const int bj = (lane & 7) + ((lane >> 3) & 1) * 8;
+  L.bc = lane >> 4;
+#pragma unroll
+  for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
+    // ranks j >= r read 16 zero bytes: their V is zero and stale weights
+    // (possibly not finite) must not meet it
+    const int j = 16 * ks + bj;
+    const bool ok = j < r;
+    L.rb[ks] = ok ? buf_u + (uint32_t)(j * wv) * 16u : zero_u;
+    L.xm[ks] = ok ? (uint32_t)(j & 7) : 0u;
+    L.cm[ks] = ok ? 0xffffffffu : 0u;
+  }
+  L.nks = (r + 15) >> 4;
+  L.ys0 = yb + g * pitch + 4 * t;
+  L.ys1 = L.ys0 + 8 * pitch;
+  L.ok0 = g < m;
+  L.ok1 = g + 8 < m;
+  return L;
+}
+
+// Staged y[row][col .. col + 1] += scale * (d0, d1) for the lane's two rows
+// (the rows go to global memory afterwards, one bulk copy each).
+__device__ __forceinline__ void expand_store(const ExpandLane &L, int col, const float (&d)[4], float scale) {
+  if (L.ok0) {
+    uint32_t *p = reinterpret_cast<uint32_t *>(L.ys0 + col * 2);
+    const uint32_t yv = *p;
+    *p = pack_bf16x2(fmaf(scale, d[0], bf16_lo(yv)), fmaf(scale, d[1], bf16_hi(yv)));
+  }
+  if (L.ok1) {
+    uint32_t *p = reinterpret_cast<uint32_t *>(L.ys1 + col * 2);
+    const uint32_t yv = *p;
+    *p = pack_bf16x2(fmaf(scale, d[2], bf16_lo(yv)), fmaf(scale, d[3], bf16_hi(yv)));
+  }
+}
+
+// G complete 16-column groups cg0, cg0 + 8, ... (their chunks lie in complete
+// groups of eight, so chunk c of rank row j sits at c ^ (j % 8)).  Each
+// group's accumulator takes, per 16-rank block, the hi term and then the lo
+// term; the G chains overlap.
+template <int JB, int G>
+__device__ __forceinline__ void expand_pass(const ExpandLane &L, const ExpandA<JB> &A, float scale, int cg0) {
   float acc[G][2][4];
 #pragma unroll
   for (int q = 0; q < G; ++q)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[q][nt][e] = 0.f;
+    for (int nt = 0; nt < 2; ++nt) acc[q][nt][0] = acc[q][nt][1] = acc[q][nt][2] = acc[q][nt][3] = 0.f;
 #pragma unroll
   for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
-    if (16 * ks >= r) break;  // rank blocks past the adapter's rank
-    // ranks j >= r read 16 zero bytes: their V is zero and stale weights
-    // (possibly not finite) must not meet it
-    const int j = 16 * ks + bj;
-    uint32_t b[G][4];
+    if (ks < L.nks) {
+      uint32_t b[G][4];
 #pragma unroll
-    for (int q = 0; q < G; ++q) {
-      if (q < ng) {
-        const int cg = cg0 + q * gstep;
-        const bool half = 2 * cg + 1 >= wv;  // an odd last chunk: only 8 columns
-        const int c = (half && bc) ? 2 * cg : 2 * cg + bc;
-        ldsm_x4_t(j < r ? wt_addr(buf_u, j, c, wv) : zero_u, b[q]);
+      for (int q = 0; q < G; ++q) {
+        const uint32_t c = (uint32_t)(2 * (cg0 + q * kConsumerWarps) + L.bc);
+        ldsm_x4_t(L.rb[ks] + (((c ^ L.xm[ks]) & L.cm[ks]) << 4), b[q]);
       }
-    }
 #pragma unroll
-    for (int q = 0; q < G; ++q) {
-      if (q < ng) {
+      for (int q = 0; q < G; ++q) {
         mma_bf16_16816(acc[q][0], A.hi[ks], b[q][0], b[q][1]);
         mma_bf16_16816(acc[q][1], A.hi[ks], b[q][2], b[q][3]);
       }
-    }
 #pragma unroll
-    for (int q = 0; q < G; ++q) {
-      if (q < ng) {
+      for (int q = 0; q < G; ++q) {
         mma_bf16_16816(acc[q][0], A.lo[ks], b[q][0], b[q][1]);
         mma_bf16_16816(acc[q][1], A.lo[ks], b[q][2], b[q][3]);
       }
@@ -319,42 +423,110 @@ __device__ __forceinline__ void expand_groups(uint32_t buf_u, const uint8_t *yb,
   }
 #pragma unroll
   for (int q = 0; q < G; ++q) {
-    if (q >= ng) break;
-    const int cg = cg0 + q * gstep;
-    const int n_nt = 2 * cg + 1 >= wv ? 1 : 2;
+    const int col = (cg0 + q * kConsumerWarps) * 16;
+    expand_store(L, col, acc[q][0], scale);
+    expand_store(L, col + 8, acc[q][1], scale);
+  }
+}
+
+// One group of a partial chunk group at the tile's end (chunks unswizzled;
+// an odd last chunk is half a group: 8 columns).
+template <int JB>
+__device__ __forceinline__ void expand_tail(const ExpandLane &L, const ExpandA<JB> &A, float scale, uint32_t zero_u,
+                                            int wv, int cg) {
+  float acc[2][4] = {};
+  const bool half = 2 * cg + 1 >= wv;
+  const uint32_t c = (uint32_t)((half && L.bc) ? 2 * cg : 2 * cg + L.bc);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      if (nt >= n_nt) break;
-      const int col = cg * 16 + nt * 8 + 2 * t;  // within the tile
+  for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
+    if (ks < L.nks) {
+      uint32_t b[4];
+      ldsm_x4_t(L.cm[ks] ? L.rb[ks] + (c << 4) : zero_u, b);
+      mma_bf16_16816(acc[0], A.hi[ks], b[0], b[1]);
+      mma_bf16_16816(acc[1], A.hi[ks], b[2], b[3]);
+      mma_bf16_16816(acc[0], A.lo[ks], b[0], b[1]);
+      mma_bf16_16816(acc[1], A.lo[ks], b[2], b[3]);
+    }
+  }
+  expand_store(L, cg * 16, acc[0], scale);
+  if (!half) expand_store(L, cg * 16 + 8, acc[1], scale);
+}
+
+// A full tile (wv = the pool's tile width): the warp's GPW column groups
+// warp, warp + 8, ... in passes of G, every B^T operand of a pass loaded
+// before its MMAs; the staged y of a group (rows 0..15, its 16 columns) is
+// read and written back with one ldmatrix / stmatrix each, in the MMA
+// fragment layout (rows past the item are staging rows nobody stores).
+template <int JB, int GPW, int G>
+__device__ __forceinline__ void expand_full(const ExpandLane &L, const ExpandA<JB> &A, float scale, uint32_t yb_u,
+                                            int pitch, int lane, int warp) {
+  // ldmatrix / stmatrix row of this lane in a group's staged y
+  const uint32_t ylane = yb_u + (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * pitch + (lane >> 4) * 16);
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int i = g + hr * 8;
-        if (i < m) {
-          const uint32_t yv = *reinterpret_cast<const uint32_t *>(yb + i * pitch + col * 2);
-          const float d0 = acc[q][nt][2 * hr], d1 = acc[q][nt][2 * hr + 1];
-          const uint32_t o = pack_bf16x2(fmaf(scale, d0, bf16_lo(yv)), fmaf(scale, d1, bf16_hi(yv)));
-          *reinterpret_cast<uint32_t *>(a.y + (long long)s_rows[i] * a.ldy + ycol + (long long)v_lo * 8 + col) = o;
+  for (int g0 = 0; g0 < GPW; g0 += G) {
+    float acc[G][2][4];
+#pragma unroll
+    for (int q = 0; q < G; ++q)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) acc[q][nt][0] = acc[q][nt][1] = acc[q][nt][2] = acc[q][nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < ExpandA<JB>::KS; ++ks) {
+      if (ks < L.nks) {
+        uint32_t b[G][4];
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+          const uint32_t c = (uint32_t)(2 * (warp + kConsumerWarps * (g0 + q)) + L.bc);
+          ldsm_x4_t(L.rb[ks] + (((c ^ L.xm[ks]) & L.cm[ks]) << 4), b[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+          mma_bf16_16816(acc[q][0], A.hi[ks], b[q][0], b[q][1]);
+          mma_bf16_16816(acc[q][1], A.hi[ks], b[q][2], b[q][3]);
+        }
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+          mma_bf16_16816(acc[q][0], A.lo[ks], b[q][0], b[q][1]);
+          mma_bf16_16816(acc[q][1], A.lo[ks], b[q][2], b[q][3]);
         }
       }
+    }
+    uint32_t yv[G][4];
+#pragma unroll
+    for (int q = 0; q < G; ++q) ldsm_x4(ylane + (uint32_t)(warp + kConsumerWarps * (g0 + q)) * 32u, yv[q]);
+#pragma unroll
+    for (int q = 0; q < G; ++q) {
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {  // e: (row g | g + 8) x (n-tile 0 | 1) as ldmatrix orders them
+        const float *d = &acc[q][e >> 1][(e & 1) * 2];
+        o[e] = pack_bf16x2(fmaf(scale, d[0], bf16_lo(yv[q][e])), fmaf(scale, d[1], bf16_hi(yv[q][e])));
+      }
+      stsm_x4(ylane + (uint32_t)(warp + kConsumerWarps * (g0 + q)) * 32u, o);
     }
   }
 }
 
-// The warp takes the 16-column groups warp, warp + 8, ..., several at a time
-// (four for ranks up to 16, two up to 32, one beyond: the larger ranks give
-// each group more MMAs of its own).
+// The warp takes the 16-column groups warp, warp + 8, ...: several at a time
+// while they lie in complete chunk groups (four for ranks up to 16, two up to
+// 32, one beyond: the larger ranks give each group more MMAs of its own),
+// then the rest one by one.
 template <int JB>
-__device__ __forceinline__ void expand_mma(uint32_t buf_u, const uint8_t *yb, uint32_t zero_u, int pitch, int wv,
-                                           int v_lo, int r, int m, const ExpandA<JB> &A, float scale,
-                                           const int *s_rows, long long ycol, const DecodeArgs &a, int lane,
-                                           int warp) {
+__device__ __forceinline__ void expand_mma(uint32_t buf_u, uint8_t *yb, uint32_t zero_u, int pitch, int wv, int r,
+                                           int m, const ExpandA<JB> &A, float scale, int lane, int warp) {
   constexpr int G = JB <= 2 ? 4 : JB == 4 ? 2 : 1;
-  const int groups = (wv + 1) / 2;  // 16-column groups (an odd last chunk is half a group)
-  for (int cg = warp; cg < groups; cg += G * kConsumerWarps) {
-    const int ng = min(G, (groups - cg + kConsumerWarps - 1) / kConsumerWarps);
-    expand_groups<JB, G>(buf_u, yb, zero_u, pitch, wv, v_lo, r, m, A, scale, s_rows, ycol, a, lane, cg,
-                         kConsumerWarps, ng);
+  const ExpandLane L = expand_lane<JB>(buf_u, yb, zero_u, pitch, wv, r, m, lane);
+  if (wv == full_tile_chunks(JB)) {
+    constexpr int GPW = full_tile_chunks(JB) / 2 / kConsumerWarps;  // column groups per warp
+    expand_full<JB, GPW, JB == 2 ? GPW : G>(L, A, scale, smem_u32(yb), pitch, lane, warp);
+    return;
   }
+  const int groups = (wv + 1) / 2;       // 16-column groups (an odd last chunk is half a group)
+  const int full = (wv & ~7) >> 1;       // groups inside complete chunk groups of eight
+  int cg = warp;
+  for (; cg + (G - 1) * kConsumerWarps < full; cg += G * kConsumerWarps) expand_pass<JB, G>(L, A, scale, cg);
+  if (G > 1)
+    for (; cg < full; cg += kConsumerWarps) expand_pass<JB, 1>(L, A, scale, cg);
+  for (; cg < groups; cg += kConsumerWarps) expand_tail<JB>(L, A, scale, zero_u, wv, cg);
 }
 
 // ------------------------------------------------------------ sync helpers
@@ -792,78 +964,112 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
   const int act_base = a.r_max * a.kcv * 16;  // activation rows follow the adapter tile
   int stage = 0;
   uint32_t phase = 0;
-  float sacc[JB < 2 ? 2 : JB][4];  // this warp's MMA fragment of the unit's V so far
-  ExpandA<JB> va;                  // the unit's V as MMA operand fragments (hi + lo)
-  while (true) {
+  // Waits for the current stage; false once the producer is done (or a wait
+  // gave up: the abort flag is then set).
+  auto acquire = [&]() -> bool {
     const bool got = cons_sync_and(mbar_wait_bounded(&S.full[stage], phase, a.status, a.wait_ns));
     if (!got) {
       if (tid == 0) set_abort(S);
-      break;
+      return false;
     }
-    const StageHdr H = S.hdr[stage];
-    const int kind = H.bits & 15;
-    if (kind == kUnitEnd) break;
-    const bool first = (H.bits >> 4) & 1, last = (H.bits >> 5) & 1;
-    const UnitRec &R = S.rec[H.bits >> 8];
-    const int m = R.m, r = R.r, wv = H.wv, v_lo = H.v_lo;
-    uint8_t *buf = S.ring + stage * a.stage_bytes;
-    const uint32_t buf_u = smem_u32(buf);
-    if (kind == kUnitShrink) {
-      if (first) {
-#pragma unroll
-        for (int nt = 0; nt < (JB < 2 ? 2 : JB); ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-      }
-      shrink_mma<JB>(buf_u, buf_u + act_base, pitch, wv, r, m, sacc, lane, warp);
-      if (last) {
-        // v of the unit's rows: the warps' fragments meet in the stage's
-        // adapter rows and are summed in fixed warp order
-        cons_sync();
-        float *red = reinterpret_cast<float *>(buf);
-        const int n = m * r;
-        shrink_spill<JB>(sacc, r, m, red + warp * kItemRows * r, lane);
-        fence_proxy_async_smem();
-        cons_sync();
-        if (MODE == kShrinkOnly) {  // to the caller: ranks r .. r_max-1 as zeros
-          for (int e = tid; e < m * a.r_max; e += kConsumerThreads) {
-            const int i = e / a.r_max, j = e - i * a.r_max;
-            float s = 0.f;
-            if (j < r) {
-#pragma unroll
-              for (int w = 0; w < kConsumerWarps; ++w) s += red[w * kItemRows * r + i * r + j];
-            }
-            a.v[(long long)R.rows[i] * a.ldv + j] = s;
-          }
-        } else {
-          for (int e = tid; e < n; e += kConsumerThreads) {
-            float s = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) s += red[w * kItemRows * r + e];
-            const int i = e / r, j = e - i * r;
-            S.v[i * a.r_max + j] = s;
-          }
-          cons_sync();
-          expand_prepare<JB>(S.v, a.r_max, r, m, va, lane);
-        }
-      }
-    } else {
-      if (MODE == kExpandOnly && first) {  // the caller's v
-        for (int e = tid; e < m * r; e += kConsumerThreads) {
-          const int i = e / r, j = e - i * r;
-          S.v[i * a.r_max + j] = a.v[(long long)R.rows[i] * a.ldv + j];
-        }
-        cons_sync();
-        expand_prepare<JB>(S.v, a.r_max, r, m, va, lane);
-      }
-      expand_mma<JB>(buf_u, buf + act_base, smem_u32(S.zero), pitch, wv, v_lo, r, m, va, R.scale, R.rows, R.ycol, a,
-                     lane, warp);
-    }
+    return (S.hdr[stage].bits & 15) != kUnitEnd;
+  };
+  auto release = [&]() {
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty[stage]);  // this warp is done with the stage
     if (++stage == NS) {
       stage = 0;
       phase ^= 1u;
     }
+  };
+  while (acquire()) {
+    StageHdr H = S.hdr[stage];
+    if ((H.bits & 15) == kUnitShrink) {
+      // the unit's shrink tiles, this one up to the one marked last; the
+      // accumulator lives only here
+      float sacc[JB < 2 ? 2 : JB][4];  // this warp's MMA fragment of the unit's V so far
+#pragma unroll
+      for (int nt = 0; nt < (JB < 2 ? 2 : JB); ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      while (true) {
+        const bool last = (H.bits >> 5) & 1;
+        const UnitRec &R = S.rec[H.bits >> 8];
+        const int m = R.m, r = R.r, wv = H.wv;
+        uint8_t *buf = S.ring + stage * a.stage_bytes;
+        const uint32_t buf_u = smem_u32(buf);
+        if (wv == full_tile_chunks(JB))
+          shrink_full<JB, full_tile_chunks(JB) / 2 / kConsumerWarps>(buf_u, buf_u + act_base, pitch, wv, r, m, sacc,
+                                                                       lane, warp);
+        else
+          shrink_mma<JB>(buf_u, buf_u + act_base, pitch, wv, r, m, sacc, lane, warp);
+        if (last) {
+          // v of the unit's rows: the warps' fragments meet in the stage's
+          // adapter rows and are summed in fixed warp order
+          cons_sync();
+          float *red = reinterpret_cast<float *>(buf);
+          const int n = m * r;
+          shrink_spill<JB>(sacc, r, m, red + warp * kItemRows * r, lane);
+          fence_proxy_async_smem();
+          cons_sync();
+          if (MODE == kShrinkOnly) {  // to the caller: ranks r .. r_max-1 as zeros
+            for (int e = tid; e < m * a.r_max; e += kConsumerThreads) {
+              const int i = e / a.r_max, j = e - i * a.r_max;
+              float s = 0.f;
+              if (j < r) {
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) s += red[w * kItemRows * r + i * r + j];
+              }
+              a.v[(long long)R.rows[i] * a.ldv + j] = s;
+            }
+          } else {
+            for (int e = tid; e < n; e += kConsumerThreads) {
+              float s = 0.f;
+#pragma unroll
+              for (int w = 0; w < kConsumerWarps; ++w) s += red[w * kItemRows * r + e];
+              const int i = e / r, j = e - i * r;
+              S.v[i * a.r_max + j] = s;
+            }
+          }
+          release();
+          break;
+        }
+        release();
+        if (!acquire()) goto done;
+        H = S.hdr[stage];
+      }
+    } else {
+      const bool first = (H.bits >> 4) & 1;
+      const UnitRec &R = S.rec[H.bits >> 8];
+      const int m = R.m, r = R.r, wv = H.wv, v_lo = H.v_lo;
+      uint8_t *buf = S.ring + stage * a.stage_bytes;
+      const uint32_t buf_u = smem_u32(buf);
+      if (MODE == kExpandOnly && first) {  // the caller's v
+        for (int e = tid; e < m * r; e += kConsumerThreads) {
+          const int i = e / r, j = e - i * r;
+          S.v[i * a.r_max + j] = a.v[(long long)R.rows[i] * a.ldv + j];
+        }
+      }
+      cons_sync();  // S.v complete (written by the shrink's last tile or just above)
+      ExpandA<JB> va;  // the unit's V as MMA operand fragments (hi + lo)
+      expand_prepare<JB>(S.v, a.r_max, r, m, va, lane);
+      uint8_t *yb = buf + act_base;
+      expand_mma<JB>(buf_u, yb, smem_u32(S.zero), pitch, wv, r, m, va, R.scale, lane, warp);
+      // the updated rows out, one bulk copy each (warp w: rows w, w + 8),
+      // before the stage is handed back
+      fence_proxy_async_smem();
+      cons_sync();
+      if (lane == 0) {
+        const long long col = R.ycol + (long long)v_lo * 8;
+        if (warp < m) bulk_s2g(a.y + (long long)R.rows[warp] * a.ldy + col, yb + warp * pitch, (uint32_t)wv * 16u);
+        if (warp + 8 < m)
+          bulk_s2g(a.y + (long long)R.rows[warp + 8] * a.ldy + col, yb + (warp + 8) * pitch, (uint32_t)wv * 16u);
+        bulk_commit();
+        bulk_wait_read();
+      }
+      release();
+    }
   }
+done:
+  if (lane == 0) bulk_wait_all();  // this warp's y rows are in global memory
 }
 
 template <int MODE, int JB>
