@@ -974,9 +974,37 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
     }
     return (S.hdr[stage].bits & 15) != kUnitEnd;
   };
+  // An expand stage goes back to the producer only once the bulk copies of
+  // its y rows have read it; with three or more stages this warp hands it
+  // back after its next tile (pend), so that the copies run during that tile.
+  int pend = -1;
   auto release = [&]() {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&S.empty[stage]);  // this warp is done with the stage
+    if (lane == 0) {
+      if (pend >= 0) {
+        bulk_wait_read();
+        mbar_arrive(&S.empty[pend]);
+      }
+      mbar_arrive(&S.empty[stage]);  // this warp is done with the stage
+    }
+    pend = -1;
+    if (++stage == NS) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  };
+  auto release_after_copies = [&]() {
+    if (NS < 3) {  // a two-stage ring: holding one back would stall the producer
+      if (lane == 0) bulk_wait_read();
+      release();
+      return;
+    }
+    __syncwarp();
+    if (lane == 0 && pend >= 0) {
+      bulk_wait_read_but_newest();  // (the previous expand stage's copies, not this one's)
+      mbar_arrive(&S.empty[pend]);
+    }
+    pend = stage;
     if (++stage == NS) {
       stage = 0;
       phase ^= 1u;
@@ -1053,8 +1081,7 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
       expand_prepare<JB>(S.v, a.r_max, r, m, va, lane);
       uint8_t *yb = buf + act_base;
       expand_mma<JB>(buf_u, yb, smem_u32(S.zero), pitch, wv, r, m, va, R.scale, lane, warp);
-      // the updated rows out, one bulk copy each (warp w: rows w, w + 8),
-      // before the stage is handed back
+      // the updated rows out, one bulk copy each (warp w: rows w, w + 8)
       fence_proxy_async_smem();
       cons_sync();
       if (lane == 0) {
@@ -1063,9 +1090,8 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
         if (warp + 8 < m)
           bulk_s2g(a.y + (long long)R.rows[warp + 8] * a.ldy + col, yb + (warp + 8) * pitch, (uint32_t)wv * 16u);
         bulk_commit();
-        bulk_wait_read();
       }
-      release();
+      release_after_copies();
     }
   }
 done:
