@@ -3,15 +3,20 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
                     [--workload q_proj|tiny|prefill|mlp|paged|qkv|swapin|linear|moe]
 
-Default workload (the metric's configuration): Llama-2-7B q_proj-shaped decode,
-d_in = d_out = 4096, rank 16 for all, 32 resident adapters in a contiguous
-stacked pool, 64 tokens with ids uniform over the 32 adapters, bf16 inputs,
-fp32 accumulation.  A step is one lora_apply call over one batch: for up to
-256 rows a single launch of the fused shrink/expand kernel, which groups the
-rows by adapter itself; beyond that the plan kernel and the delta kernel.
-Steps rotate over up to 64 independent buffer sets (pool, x, y, ids,
-workspace), > 4x the 126 MB L2, so every step reads its adapters and
-activations from HBM.
+Default workload: the largest single-GPU configuration, the S-LoRA-style
+paged step -- 1000 rank-16 adapters on q/k/v/o of 32 layers at hidden 4096
+(a 31.25 GiB pool of 1 MiB pages scattered by a seeded permutation), a decode
+batch of 512 tokens over 64 distinct adapters drawn Zipf(1.1), and all 128
+layer x projection deltas per step: one plan (lora_plan_ids) and 128
+lora_apply_plan calls, bf16 inputs, fp32 accumulation.  The pool and the
+step's 1 GiB of activations exceed the 126 MB L2, so every matrix reads its
+adapters and activations from HBM.
+
+Other workloads (--workload): q_proj (Llama-2-7B q_proj-shaped decode,
+d_in = d_out = 4096, rank 16, 32 adapters in a contiguous pool, 64 tokens;
+one fused launch per batch; steps rotate over up to 64 buffer sets, > 4x the
+L2), tiny, prefill (segmented tensor-core path), mlp (mixed ranks padded to
+64, 4096 -> 11008), qkv, linear, moe and swapin.
 
 Printed: one JSON line (rank 0).  value = tokens/s over all ranks; roofline =
 algorithmic bytes of the dominant kernel / its mean launch time (CUDA events
@@ -481,10 +486,13 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
 
     import adapter_deltas_b200 as L
     T, n_t = w.T, len(w.targets)
-    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, w.n_slots, w.page_bytes)
+    active = [int(s) for s in w.active_slots]
+    # --pool active: pages for the batch's active slots only (a few GB, for
+    # profiler captures); the kernels read the same bytes per matrix
+    n_pages_slots = len(active) if args.pool == "active" else w.n_slots
+    pool_bytes = L.lora_pool_bytes_required(w.targets, w.r_max, n_pages_slots, w.page_bytes)
     mem = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
     pool = L.lora_pool_create(dev.index, w.targets, w.r_max, w.n_slots, w.page_bytes, mem, w.scatter_seed)
-    active = [int(s) for s in w.active_slots]
     w.prefetch(active, range(n_t))
     for s in active:
         for t in range(n_t):
@@ -493,8 +501,9 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
     g = torch.Generator(device=dev).manual_seed(7)
     fa = (torch.randn(16, 4096, generator=g, device=dev) / 64).to(torch.bfloat16)
     fb = (torch.randn(4096, 16, generator=g, device=dev) * 0.14).to(torch.bfloat16)
-    for s in range(w.n_slots):
-        if s not in set(active):
+    act = set(active)
+    for s in range(w.n_slots if args.pool == "full" else 0):
+        if s not in act:
             for t in range(n_t):
                 L.lora_pool_load(pool, s, t, 16, fa, fb)
     xs = [bf16(w.x(t)) for t in range(n_t)]
@@ -580,7 +589,10 @@ def run_paged(args, rank, world, dev, w, scales, bf16):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": T * world, "seq_len": 1,
                    "parallelism": "replicas%d" % world if world > 1 else "single",
-                   "deltas_per_step": n_t, "l2": "pool 31.25 GiB and 1 GiB of activations per step > L2",
+                   "deltas_per_step": n_t,
+                   "pool": ("31.25 GiB, every slot loaded" if args.pool == "full"
+                            else "pages of the %d active slots only" % len(active)),
+                   "l2": "pool and 1 GiB of activations per step > L2",
                    "timing": "CUDA graph of the K steps, CUDA events around its replay"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind, "traffic": traffic_from_profile("decode_kernel", "decode.cu", "paged"),
@@ -1167,11 +1179,13 @@ def job_value(tokens_per_rank: int, world: int, ms_max: float) -> float:
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--workload", default="q_proj", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="paged", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--pool", default="full", choices=["full", "active"],
+                    help="paged workload: a pool for all 1000 slots, or pages for the active slots only")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
