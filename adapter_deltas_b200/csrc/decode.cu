@@ -49,6 +49,9 @@ constexpr int dec_min_blocks(int jb) { return jb == 2 ? 1 : 2; }
 // 16-byte chunks per row of a full pool tile for the kernel's rank class
 // (the tile width of the largest rank the class serves).
 __host__ __device__ constexpr int full_tile_chunks(int jb) { return pool_tile_cols(8 * jb) / 8; }
+// Items of up to this many rows write their y rows back with plain stores;
+// larger ones with bulk copies.
+constexpr int kStoreRowsMax = 4;
 constexpr int kCacheItems = 256;  // items whose records a CTA keeps in shared memory
 constexpr int kCachePerm = 512;   // grouped row positions a CTA keeps in shared memory
 
@@ -1081,17 +1084,31 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
       expand_prepare<JB>(S.v, a.r_max, r, m, va, lane);
       uint8_t *yb = buf + act_base;
       expand_mma<JB>(buf_u, yb, smem_u32(S.zero), pitch, wv, r, m, va, R.scale, lane, warp);
-      // the updated rows out, one bulk copy each (warp w: rows w, w + 8)
-      fence_proxy_async_smem();
-      cons_sync();
-      if (lane == 0) {
-        const long long col = R.ycol + (long long)v_lo * 8;
-        if (warp < m) bulk_s2g(a.y + (long long)R.rows[warp] * a.ldy + col, yb + warp * pitch, (uint32_t)wv * 16u);
-        if (warp + 8 < m)
-          bulk_s2g(a.y + (long long)R.rows[warp + 8] * a.ldy + col, yb + (warp + 8) * pitch, (uint32_t)wv * 16u);
-        bulk_commit();
+      // the updated rows out (warp w: rows w, w + 8).  A few rows: the
+      // warp's lanes store consecutive 16-byte chunks (whole lines per
+      // instruction) and the stage goes back at once.  More: one bulk copy
+      // per row, the stage handed back once the copies have read it.
+      if (m <= kStoreRowsMax) {
+        cons_sync();
+        for (int i = warp; i < m; i += kConsumerWarps) {
+          const uint8_t *src = yb + i * pitch;
+          uint16_t *dst = a.y + (long long)R.rows[i] * a.ldy + R.ycol + (long long)v_lo * 8;
+          for (int ch = lane; ch < wv; ch += 32)
+            *reinterpret_cast<uint4 *>(dst + ch * 8) = *reinterpret_cast<const uint4 *>(src + ch * 16);
+        }
+        release();
+      } else {
+        fence_proxy_async_smem();
+        cons_sync();
+        if (lane == 0) {
+          const long long col = R.ycol + (long long)v_lo * 8;
+          if (warp < m) bulk_s2g(a.y + (long long)R.rows[warp] * a.ldy + col, yb + warp * pitch, (uint32_t)wv * 16u);
+          if (warp + 8 < m)
+            bulk_s2g(a.y + (long long)R.rows[warp + 8] * a.ldy + col, yb + (warp + 8) * pitch, (uint32_t)wv * 16u);
+          bulk_commit();
+        }
+        release_after_copies();
       }
-      release_after_copies();
     }
   }
 done:
