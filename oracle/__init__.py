@@ -88,7 +88,7 @@ def _load():
     lib.oracle_linear.restype = None
     lib.oracle_linear.argtypes = [I, I, I, P, P, P, I]
     lib.oracle_lora_params.restype = ctypes.c_longlong
-    lib.oracle_lora_params.argtypes = [ctypes.c_longlong] * 4
+    lib.oracle_lora_params.argtypes = [I, P, P, ctypes.c_longlong, ctypes.c_longlong]
     _lib = lib
     return lib
 
@@ -288,7 +288,14 @@ def slot_layout(targets: Sequence[Tuple[int, int]], r_max: int):
     return a_off, bt_off, int(total)
 
 
-def lora_params(hidden: int = 4096, layers: int = 32, rank: int = 16,
-                n_targets: int = 4) -> int:
-    """r * (d_in + d_out) per square matrix, times targets, times layers."""
-    return int(_load().oracle_lora_params(hidden, layers, rank, n_targets))
+ATTENTION_4096 = ((4096, 4096),) * 4   # q, k, v, o projections of Llama-2-7B (d_in, d_out)
+
+
+def lora_params(shapes=ATTENTION_4096, layers: int = 32, rank: int = 16) -> int:
+    """Parameters of a rank-`rank` adapter on the matrices `shapes` ((d_in,
+    d_out) per adapted matrix of one layer) in each of `layers` layers: A is
+    r x d_in and B is d_out x r for each matrix."""
+    lib = _load()
+    d_in = np.array([s[0] for s in shapes], dtype=np.int64)
+    d_out = np.array([s[1] for s in shapes], dtype=np.int64)
+    return int(lib.oracle_lora_params(len(shapes), _ptr(d_in), _ptr(d_out), layers, rank))

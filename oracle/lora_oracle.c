@@ -339,12 +339,19 @@ long long oracle_slot_layout(int n_targets, const int32_t *d_in,
 /* ---------------------------------------------------------------------- */
 
 /*
- * Parameter count of a rank-r adapter on n_targets square hidden x hidden
- * matrices in each of n_layers layers: r * (d_in + d_out) per matrix.
+ * Parameter count of a rank-r adapter.  An adapted matrix W of shape
+ * d_out x d_in gets A (r x d_in) and B (d_out x r): r d_in + d_out r
+ * parameters.  A layer adapts n_targets matrices (shapes d_in[t] x d_out[t]);
+ * the adapter covers n_layers such layers.
  */
-long long oracle_lora_params(long long hidden, long long n_layers,
-                             long long rank, long long n_targets)
+long long oracle_lora_params(int n_targets, const long long *d_in, const long long *d_out,
+                             long long n_layers, long long rank)
 {
-    long long per_matrix = rank * (hidden + hidden);
-    return per_matrix * n_targets * n_layers;
+    long long per_layer = 0;
+    for (int t = 0; t < n_targets; ++t) {
+        long long a_params = rank * d_in[t];   /* A */
+        long long b_params = d_out[t] * rank;  /* B */
+        per_layer += a_params + b_params;
+    }
+    return per_layer * n_layers;
 }

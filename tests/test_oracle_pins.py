@@ -56,8 +56,8 @@ def _rand_case(seed, T, d_in, d_out, ranks, alphas, none_frac=0.25):
 
 def test_sizing_matches_printed_example():
     g = _golden("lora_sizing.txt")
-    params = oracle.lora_params(int(g["hidden"]), int(g["layers"]), int(g["rank"]),
-                                int(g["targets"]))
+    h = int(g["hidden"])
+    params = oracle.lora_params(((h, h),) * int(g["targets"]), int(g["layers"]), int(g["rank"]))
     nbytes = params * int(g["dtype_bytes"])
     assert f"{params / 1e6:.1f}M params, {nbytes / 2**20:.1f} MiB" == g["printed"]
     # closed form: 16 * 8192 * 4 * 32 = 2^24 parameters, exactly 32 MiB
@@ -67,17 +67,33 @@ def test_sizing_matches_printed_example():
 
 
 def test_sizing_scales_with_rank_and_targets():
-    base = oracle.lora_params(4096, 32, 16, 4)
-    assert oracle.lora_params(4096, 32, 32, 4) == 2 * base      # doubling rank doubles bytes
-    assert oracle.lora_params(4096, 32, 16, 8) == 2 * base
-    assert oracle.lora_params(4096, 1, 1, 1) == 8192             # r (d_in + d_out)
+    att = ((4096, 4096),) * 4
+    base = oracle.lora_params(att, 32, 16)
+    assert oracle.lora_params(att, 32, 32) == 2 * base           # doubling rank doubles bytes
+    assert oracle.lora_params(att * 2, 32, 16) == 2 * base       # twice the matrices
+    assert oracle.lora_params(((4096, 4096),), 1, 1) == 8192     # r (d_in + d_out)
+    assert oracle.lora_params(((3, 5),), 1, 1) == 8              # A 1 x 3, B 5 x 1
+    assert oracle.lora_params(((3, 5),), 7, 2) == 7 * 2 * 8       # linear in layers and rank
+
+
+def test_sizing_of_the_mlp_projections():
+    # The same page adds gate/up/down (d_ff = 11008 on Llama-2-7B): each of
+    # those matrices is r (4096 + 11008) parameters.  The page calls the
+    # result roughly 4x the attention-only adapter; r (d_in + d_out) gives
+    # (4 * 8192 + 3 * 15104) / (4 * 8192) = 2.38x -- the formula decides.
+    att = ((4096, 4096),) * 4
+    mlp = ((4096, 11008), (4096, 11008), (11008, 4096))
+    assert oracle.lora_params(mlp, 1, 16) == 3 * 16 * 15104
+    both = oracle.lora_params(att + mlp, 32, 16)
+    assert both == 32 * 16 * (4 * 8192 + 3 * 15104)
+    assert round(both / oracle.lora_params(att, 32, 16), 2) == 2.38
 
 
 def test_slot_layout_of_the_paged_geometry_is_the_adapter_size():
     # 32 layers x q/k/v/o at hidden 4096, rank 16: one slot is exactly the
     # printed adapter size, and each target block starts 256 KiB after the last.
     a_off, bt_off, total = oracle.slot_layout([(4096, 4096)] * 128, 16)
-    assert total == oracle.lora_params(4096, 32, 16, 4) * 2
+    assert total == oracle.lora_params(((4096, 4096),) * 4, 32, 16) * 2
     assert np.array_equal(a_off, np.arange(128) * 256 * 1024)
     assert np.array_equal(bt_off, np.arange(128) * 256 * 1024 + 128 * 1024)
 
