@@ -97,6 +97,7 @@ _sig("lora_apply_noalloc", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
 _sig("lora_get_error", _I, [_P, ctypes.POINTER(_I), _P])
 _sig("lora_kernel_launches", ctypes.c_uint64, [])
 _sig("lora_set_wait_limit_ns", None, [ctypes.c_uint64])
+_sig("lora_selftest_stalled_apply", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P])
 
 
 class LoraError(RuntimeError):
@@ -357,3 +358,11 @@ def lora_kernel_launches() -> int:
 def lora_set_wait_limit_ns(ns: int) -> None:
     """Wall-clock limit of the decode kernel's bounded waits (0: one second)."""
     _lib.lora_set_wait_limit_ns(int(ns))
+
+
+def lora_selftest_stalled_apply(pool: PoolHandle, target: int, x, y, ids, scales, stream=None) -> None:
+    """Test only: the decode launch of lora_apply with no stage ever filled,
+    so that its waits run out (LORA_ERR_TIMEOUT in the sticky status)."""
+    _check(_lib.lora_selftest_stalled_apply(pool, target, _ptr(x), _ld(x), _ptr(y), _ld(y), _ptr(ids),
+                                            _ptr(scales), y.shape[0], _stream(stream)),
+           "lora_selftest_stalled_apply")

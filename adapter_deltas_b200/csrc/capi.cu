@@ -177,6 +177,29 @@ int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ld
   return lora_apply_plan(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, stream);
 }
 
+int lora_selftest_stalled_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
+                                const int32_t *ids, const float *scales, int T, void *stream) {
+  if (!p || target < 0 || target >= p->n_targets || T < 0 || T > kFusedMaxT) return LORA_ERR_INVALID_ARG;
+  if (T == 0) return LORA_OK;
+  int rc;
+  if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
+  if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
+  if (!scales || !ids) return LORA_ERR_INVALID_ARG;
+  if (overlap(x, ldx, y, ldy, T)) return LORA_ERR_INVALID_ARG;
+  DeviceGuard g(p->device);
+  DecodeCall c;
+  c.targets = &target;
+  c.x = x;
+  c.ldx = ldx;
+  c.y = y;
+  c.ldy = ldy;
+  c.scales = scales;
+  c.T = T;
+  c.ids = ids;
+  c.stall = 1;
+  return launch_decode(p, c, static_cast<cudaStream_t>(stream));
+}
+
 int lora_apply_multi(lora_pool *p, int n_targets, const int *targets, const void *x, int ldx, void *y, int ldy,
                      const int *y_cols, const int32_t *ids, const float *scales, int T, void *ws, size_t ws_bytes,
                      void *stream) {

@@ -105,6 +105,7 @@ struct DecodeArgs {
   int moe_k, moe_e;
   float *v;  // shrink-only: output [T, ldv]; expand-only: input
   long long ldv;
+  int stall;  // test only: the producer fills no stage
   int *status;
   unsigned long long wait_ns;
   int kcv;        // 16-byte chunks per full tile row (the pool's tile width)
@@ -838,6 +839,7 @@ __device__ __forceinline__ void set_abort(const DecSmem &S) { *(volatile int *)S
 // the copies.
 template <int MODE, int JB>
 __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int lane) {
+  if (a.stall) return;  // (test of the bounded waits: the consumers' first wait runs out)
   const UnitGeo<MODE> U(a, n_items);
   const int NS = a.n_stages, NT = a.n_tgt;
   const bool fused = a.ids != nullptr;
@@ -1288,6 +1290,7 @@ int launch_decode(lora_pool *pool, const DecodeCall &c, cudaStream_t st) {
   a.moe_e = c.moe_e;
   a.v = c.v;
   a.ldv = c.ldv;
+  a.stall = c.stall;
   a.status = pool->d_status;
   a.wait_ns = g_wait_ns.load();
   const DecodeGeo g = decode_geometry(pool->r_max);

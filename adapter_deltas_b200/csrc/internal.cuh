@@ -420,6 +420,7 @@ struct DecodeCall {
   int x_div = 1;
   const int32_t *moe_topk = nullptr;
   int moe_k = 0, moe_e = 0;
+  int stall = 0;  // test only: the producer fills no stage, so every consumer wait runs out
 };
 int launch_decode(lora_pool *pool, const DecodeCall &c, cudaStream_t st);
 // Lowers (ns > 0) or restores (0) the wall-clock limit of the decode

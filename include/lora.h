@@ -299,7 +299,29 @@ LORA_API int lora_apply_plan(lora_pool *pool, int target, const void *x, int ldx
 /* ------------------------------------------------------- one-call entry */
 
 /*
- * lora_plan_ids followed by lora_apply_plan, with the same result.  Batches
+ * The heterogeneous-batch delta: for every row t with a = ids[t] != -1,
+ *     y[t] += scales[a] * B_a (A_a x[t]),
+ * the per-request term of y = xW + (x A) B (alpha / r) on "Multi-LoRA
+ * Serving: Why 100 Adapters Fit on One GPU" (section "Why can't you just
+ * merge LoRA weights into the base model?"; A_a here holds the rows of that
+ * page's A transposed, so A_a x[t] is its x A), computed for every adapter of
+ * the batch in one call from an index vector and the stacked pool, as the
+ * same page's section "How does one batch run 30 different adapters at
+ * once?" describes; xW is the caller's (y on entry).
+ *   x, ldx   device bf16 [T, ldx], ldx >= d_in, a multiple of 8, 16-byte
+ *            aligned; read only; must not overlap y
+ *   y, ldy   device bf16 [T, ldy], ldy >= d_out, a multiple of 8, 16-byte
+ *            aligned; each adapted element becomes bf16_rn(y + scale *
+ *            delta) computed in fp32; rows with id -1 are not touched
+ *   ids      device int32 [T]: slot of each row, -1 = no adapter
+ *   scales   device fp32 [n_slots]: alpha / r of each slot's adapter
+ *   ws       device workspace of at least lora_workspace_bytes(pool, target,
+ *            T) bytes, 16-byte aligned (caller-owned)
+ * Errors: host-checked arguments return LORA_ERR_INVALID_ARG /
+ * LORA_ERR_ALIGNMENT / LORA_ERR_WORKSPACE with nothing launched; bad ids
+ * and unloaded slots found on the device leave their rows untouched and set
+ * the sticky status (lora_get_error).
+ * Same result as lora_plan_ids followed by lora_apply_plan.  Batches
  * of at most 256 rows take one launch instead: the delta kernel groups the
  * rows itself (the same segments and items as lora_plan_ids), and ws is then
  * not written -- callers that reuse a plan across targets call lora_plan_ids
@@ -422,14 +444,26 @@ LORA_API int lora_linear_expand(lora_pool *pool, int target, const void *x, int 
  * arguments). */
 LORA_API size_t lora_linear_workspace_bytes(const lora_pool *pool, int target, int max_tokens);
 
-/* lora_plan_segments followed by lora_apply_plan. */
+/*
+ * The delta for a batch given as contiguous segments (rows seg_offsets[s] ..
+ * seg_offsets[s+1]-1 use slot seg_slot[s]): the segmented gather-and-multiply
+ * of "Multi-LoRA Serving: Why 100 Adapters Fit on One GPU", section "How does
+ * one batch run 30 different adapters at once?", whose last paragraph notes
+ * that prefill is compute-bound -- long segments therefore run on the tensor
+ * cores, short ones on the decode kernel.  Arguments as lora_plan_segments
+ * and lora_apply_plan; the result is that of lora_plan_segments followed by
+ * lora_apply_plan.
+ */
 LORA_API int lora_apply_segments(lora_pool *pool, int target, const void *x, int ldx,
                         void *y, int ldy, const int32_t *seg_offsets,
                         const int32_t *seg_slot, int S, const float *scales,
                         int T, void *ws, size_t ws_bytes, void *stream);
 
 /*
- * The two halves of the delta, for callers that keep v = A_a x[t]:
+ * The two halves of the delta -- the adapter "shrink" (v = A_a x, rank r_a
+ * out of d_in) and "expand" (y += scale B_a v) steps that "Multi-LoRA
+ * Serving: Sharing One GPU Across Adapters" names in its section "MoE Models
+ * Raise the Bar" -- for callers that keep v = A_a x[t]:
  *   lora_shrink writes v[t, 0:r_max] (fp32, device [T, ldv], ldv >= r_max;
  *   entries r_a..r_max-1 are written as 0) for every row with an adapter,
  *   and leaves other rows of v untouched.
@@ -484,8 +518,16 @@ LORA_API int lora_apply_noalloc(lora_pool *pool, int target, const void *x, int 
 
 /* ------------------------------------------------------------ diagnostics */
 
-/* Synchronise stream, then read and clear the pool's sticky device status
- * (LORA_OK when no device-side error happened since the last read). */
+/*
+ * Synchronise stream, then read and clear the pool's sticky device status
+ * (LORA_OK when no device-side error happened since the last read) into
+ * *device_status.  The pages define no error channel; this one is the
+ * library's own: device-side checks (an id outside [-1, n_slots), a slot
+ * not loaded, a bounded wait that ran out) never fault, they record their
+ * code here (the first one wins) and leave the affected rows untouched.
+ * Returns LORA_ERR_INVALID_ARG for a null pool or device_status,
+ * LORA_ERR_CUDA if the synchronisation fails.
+ */
 LORA_API int lora_get_error(lora_pool *pool, int *device_status, void *stream);
 
 /* Number of kernels this library has launched in this process. */
@@ -493,13 +535,26 @@ LORA_API uint64_t lora_kernel_launches(void);
 
 /*
  * Wall-clock limit of the decode kernel's bounded waits (for a stage of its
- * copy ring, or for the shrink partials of an item), in nanoseconds, for the
- * launches that follow; 0 restores the default of one second.  A wait that
+ * copy ring), in nanoseconds, for the launches that follow; 0 restores the default of one second.  A wait that
  * runs out sets LORA_ERR_TIMEOUT in the pool's sticky status, leaves the
  * rows that needed the data untouched and lets the kernel finish; it never
  * faults.  Tests lower it to reach that path quickly.
  */
 LORA_API void lora_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Test of the bounded waits (no use outside tests).  Launches the decode
+ * kernel of lora_apply for a batch of T <= 256 rows (arguments as for
+ * lora_apply; no workspace) with its copy warp told to fill no stage, so
+ * that the compute warps' first wait runs out after the limit set by
+ * lora_set_wait_limit_ns.  Expected outcome: the launch completes,
+ * lora_get_error then reads LORA_ERR_TIMEOUT, and y is left as it was.  No
+ * copy is in flight when the wait gives up, and the CUDA context stays
+ * usable.  Returns LORA_ERR_INVALID_ARG for T > 256.
+ */
+LORA_API int lora_selftest_stalled_apply(lora_pool *pool, int target, const void *x, int ldx,
+                                void *y, int ldy, const int32_t *ids,
+                                const float *scales, int T, void *stream);
 
 #ifdef __cplusplus
 }
