@@ -571,6 +571,7 @@ struct DecSmem {
   int4 *c_item;           // [kCacheItems]: slot, first grouped position, rows
   int4 *c_slot;           // [kCacheItems]: rank, A page, B^T page, scale bits (first target)
   int *c_perm;            // [kCachePerm]: row of each grouped position
+  long long *tg;          // [3][kMaxMulti]: the launch's targets' A offset, B^T offset, first y column
   // in-kernel grouping temporaries, inside the ring (unused until the
   // grouping is done)
   int *g_key;        // [kGroupTable] hash table of the batch's slots (-1: empty)
@@ -589,7 +590,7 @@ constexpr int kRingMin = 40 * 1024;  // room for the grouping temporaries
 
 constexpr int dec_extra_bytes(int r_max) {
   return kMaxStages * (int)sizeof(StageHdr) + kRecs * (int)sizeof(UnitRec) + 2 * kMaxStages * 8 + 64 +
-         kItemRows * r_max * 4 + 64 + kCacheItems * 32 + kCachePerm * 4;
+         kItemRows * r_max * 4 + 64 + kCacheItems * 32 + kCachePerm * 4 + 3 * kMaxMulti * 8;
 }
 
 __device__ __forceinline__ DecSmem dec_carve(uint8_t *smem, const DecodeArgs &a) {
@@ -605,7 +606,8 @@ __device__ __forceinline__ DecSmem dec_carve(uint8_t *smem, const DecodeArgs &a)
   S.misc = reinterpret_cast<int *>(p); p += 64;
   S.c_item = reinterpret_cast<int4 *>(p); p += kCacheItems * 16;
   S.c_slot = reinterpret_cast<int4 *>(p); p += kCacheItems * 16;
-  S.c_perm = reinterpret_cast<int *>(p);
+  S.c_perm = reinterpret_cast<int *>(p); p += kCachePerm * 4;
+  S.tg = reinterpret_cast<long long *>(p);
   uint8_t *q = S.ring;
   S.g_key = reinterpret_cast<int *>(q); q += kGroupTable * 4;
   S.g_cnt = reinterpret_cast<int *>(q); q += kGroupTable * kConsumerWarps * 4;
@@ -675,8 +677,11 @@ __device__ int fused_group(const DecodeArgs &a, const DecSmem &S, int tid) {
   for (int i = tid; i < kGroupTable; i += kDecThreads) S.g_key[i] = -1;
   for (int i = tid; i < kGroupTable * kConsumerWarps; i += kDecThreads) S.g_cnt[i] = 0;
   for (int i = tid; i < n_words; i += kDecThreads) S.g_bits[i] = 0u;
-  int key = -1, bad = 0, empty = 0;
-  int4 sinfo = make_int4(0, -1, -1, 0);
+  // The slot's record loads stay in flight through the grouping: only the
+  // thread that records an item uses them.  A slot that is not loaded still
+  // forms its items; they get rank 0 and are skipped (rows untouched).
+  int key = -1, bad = 0;
+  int ld = 1, rk = 0, pa = -1, pb = -1, sc = 0;
   if (tid < T) {
     const int id = a.moe_topk ? moe_pair_slot(a, tid) : a.ids[tid];
     if (id != -1) {
@@ -684,25 +689,18 @@ __device__ int fused_group(const DecodeArgs &a, const DecSmem &S, int tid) {
         bad = 1;
       } else {
         const PoolView &p = a.pool;
-        const int ld = p.loaded[id];
-        const int rk = p.rank[(long long)id * p.n_targets + a.tgt[0]];
-        const int pa = block_page(p, id, a.a_off[0], (long long)a.r_max * a.d_in * 2);
-        const int pb = block_page(p, id, a.bt_off[0], (long long)a.r_max * a.d_out * 2);
-        const int sc = a.scales ? __float_as_int(a.scales[id]) : 0;
-        if (ld) {
-          key = id;
-          sinfo = make_int4(rk, pa, pb, sc);
-        } else {
-          empty = 1;
-        }
+        key = id;
+        ld = p.loaded[id];
+        rk = p.rank[(long long)id * p.n_targets + a.tgt[0]];
+        pa = block_page(p, id, a.a_off[0], (long long)a.r_max * a.d_in * 2);
+        pb = block_page(p, id, a.bt_off[0], (long long)a.r_max * a.d_out * 2);
+        sc = a.scales ? __float_as_int(a.scales[id]) : 0;
       }
     }
   }
   const int any_bad = __syncthreads_or(bad);  // (also orders the clearing above before the inserts)
-  const int any_empty = __syncthreads_or(empty);
   if (blockIdx.x == 0 && tid == 0) {
     if (any_bad) set_status(a.status, LORA_ERR_BAD_ID);
-    else if (any_empty) set_status(a.status, LORA_ERR_NOT_LOADED);
   }
   // (1) the slot into the hash table (at most kFusedMaxT keys in twice as
   // many entries) and the bitmap
@@ -773,10 +771,11 @@ __device__ int fused_group(const DecodeArgs &a, const DecSmem &S, int tid) {
     if (local % kItemRows == 0) {
       const int item = S.g_ditem[d] + local / kItemRows;
       S.c_item[item] = make_int4(key, pos, min(kItemRows, S.g_dtot[d] - local), 0);
-      S.c_slot[item] = sinfo;
+      S.c_slot[item] = ld ? make_int4(rk, pa, pb, sc) : make_int4(0, -1, -1, 0);
     }
   }
-  __syncthreads();
+  const int any_empty = __syncthreads_or(key >= 0 && !ld);
+  if (blockIdx.x == 0 && tid == 0 && !any_bad && any_empty) set_status(a.status, LORA_ERR_NOT_LOADED);
   return items_tot;
 }
 
@@ -909,15 +908,15 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
     // lane L (1 <= L <= m) copies activation row L - 1: its x row and y row
     const int arow = __shfl_sync(0xffffffffu, myrow, (lane + 31) & 31);
     const uint8_t *x_row = reinterpret_cast<const uint8_t *>(a.x + (long long)(arow / a.x_div) * a.ldx);
-    const uint8_t *y_row = reinterpret_cast<const uint8_t *>(a.y + (long long)arow * a.ldy + a.y_col[ti]);
-    const long long a_blk = a.a_off[ti], b_blk = a.bt_off[ti];
+    const long long a_blk = S.tg[ti], b_blk = S.tg[kMaxMulti + ti], ycol = S.tg[2 * kMaxMulti + ti];
+    const uint8_t *y_row = reinterpret_cast<const uint8_t *>(a.y + (long long)arow * a.ldy + ycol);
     // ---- the unit's record (its ring slot is free: every stage that named
     // it NS + 1 records ago has been released by now)
     UnitRec &R = S.rec[rec];
     if (lane == 0) {
       R.m = m;
       R.r = r;
-      R.ycol = (int)a.y_col[ti];
+      R.ycol = (int)ycol;
       R.scale = scale;
     }
     if (lane < kItemRows) R.rows[lane] = myrow;
@@ -1131,6 +1130,11 @@ __global__ void __launch_bounds__(kDecThreads, dec_min_blocks(JB)) decode_kernel
     fence_mbar_init();
   }
   if (tid < 16) reinterpret_cast<uint32_t *>(S.zero)[tid] = 0u;
+  if (tid < kMaxMulti) {  // (kernel parameters: read while the previous launch may still run)
+    S.tg[tid] = a.a_off[tid];
+    S.tg[kMaxMulti + tid] = a.bt_off[tid];
+    S.tg[2 * kMaxMulti + tid] = a.y_col[tid];
+  }
   __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
