@@ -390,7 +390,7 @@ struct DeviceGuard {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Launchers (defined in plan.cu / sgmv.cu).
+// Launchers (defined in plan.cu / decode.cu).
 int launch_plan_ids(lora_pool *pool, const int32_t *ids, int T, void *ws, cudaStream_t st);
 int launch_plan_segments(lora_pool *pool, const int32_t *off, const int32_t *slot, int S, int T,
                          void *ws, cudaStream_t st);
