@@ -105,6 +105,7 @@ struct DecodeArgs {
   int moe_k, moe_e;
   float *v;  // shrink-only: output [T, ldv]; expand-only: input
   long long ldv;
+  int n_sms;  // SMs of the device
   int stall;  // test only: the producer fills no stage
   int *status;
   unsigned long long wait_ns;
@@ -571,6 +572,7 @@ struct DecSmem {
   int4 *c_item;           // [kCacheItems]: slot, first grouped position, rows
   int4 *c_slot;           // [kCacheItems]: rank, A page, B^T page, scale bits (first target)
   int *c_perm;            // [kCachePerm]: row of each grouped position
+  int *c_pref;            // [kCacheItems + 1]: column ranges of the items before each (uneven ranges)
   long long *tg;          // [3][kMaxMulti]: the launch's targets' A offset, B^T offset, first y column
   // in-kernel grouping temporaries, inside the ring (unused until the
   // grouping is done)
@@ -590,7 +592,8 @@ constexpr int kRingMin = 40 * 1024;  // room for the grouping temporaries
 
 constexpr int dec_extra_bytes(int r_max) {
   return kMaxStages * (int)sizeof(StageHdr) + kRecs * (int)sizeof(UnitRec) + 2 * kMaxStages * 8 + 64 +
-         kItemRows * r_max * 4 + 64 + kCacheItems * 32 + kCachePerm * 4 + 3 * kMaxMulti * 8;
+         kItemRows * r_max * 4 + 64 + kCacheItems * 32 + kCachePerm * 4 + 3 * kMaxMulti * 8 +
+         (kCacheItems + 4) * 4;
 }
 
 __device__ __forceinline__ DecSmem dec_carve(uint8_t *smem, const DecodeArgs &a) {
@@ -607,7 +610,8 @@ __device__ __forceinline__ DecSmem dec_carve(uint8_t *smem, const DecodeArgs &a)
   S.c_item = reinterpret_cast<int4 *>(p); p += kCacheItems * 16;
   S.c_slot = reinterpret_cast<int4 *>(p); p += kCacheItems * 16;
   S.c_perm = reinterpret_cast<int *>(p); p += kCachePerm * 4;
-  S.tg = reinterpret_cast<long long *>(p);
+  S.tg = reinterpret_cast<long long *>(p); p += 3 * kMaxMulti * 8;
+  S.c_pref = reinterpret_cast<int *>(p);
   uint8_t *q = S.ring;
   S.g_key = reinterpret_cast<int *>(q); q += kGroupTable * 4;
   S.g_cnt = reinterpret_cast<int *>(q); q += kGroupTable * kConsumerWarps * 4;
@@ -830,6 +834,38 @@ struct UnitGeo {
 __device__ __forceinline__ bool aborted(const DecSmem &S) { return *(volatile int *)S.misc != 0; }
 __device__ __forceinline__ void set_abort(const DecSmem &S) { *(volatile int *)S.misc = 1; }
 
+// Uneven column ranges (the copy warp; every CTA computes the same).  An
+// item's expand tiles carry its rows of y in and out, so an item of many rows
+// costs its CTA far more than a small one.  When the uniform split leaves
+// SMs without a unit, each item of more than kSmallRows rows gets twice the
+// uniform number of column ranges (at most one per expand tile), provided
+// the units still fit one per SM; each of its units recomputes the item's
+// shrink.  Returns the unit count (0: keep the uniform split) and writes the
+// exclusive prefix of the items' range counts to S.c_pref.
+constexpr int kSmallRows = 4;
+__device__ int uneven_ranges(const DecodeArgs &a, const DecSmem &S, int n_items, int nnu, int nnt, int lane) {
+  if (n_items > kCacheItems || (long long)n_items * nnu * a.n_tgt >= (long long)a.n_sms) return 0;
+  const int big_k = min(2 * nnu, nnt);
+  if (big_k == nnu) return 0;
+  int base = 0;
+  for (int t0 = 0; t0 < n_items; t0 += 32) {
+    const int t = t0 + lane;
+    const int k = t < n_items ? (S.c_item[t].z > kSmallRows ? big_k : nnu) : 0;
+    int inc = k;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += v;
+    }
+    if (t < n_items) S.c_pref[t] = base + inc - k;
+    base += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  if (base == n_items * nnu || (long long)base * a.n_tgt > (long long)a.n_sms) return 0;  // nothing to gain
+  if (lane == 0) S.c_pref[n_items] = base;
+  __syncwarp();
+  return base * a.n_tgt;
+}
+
 // Producer warp: walks the CTA's units (blockIdx.x, + gridDim.x, ...) and
 // copies their tiles into the ring -- rows 0 .. r-1 of an adapter tile as one
 // bulk copy (one contiguous range of the pool block), then one bulk copy per
@@ -867,16 +903,39 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
       ++round;
     }
   };
+  const int n_uneven = MODE == kFused ? uneven_ranges(a, S, n_items, U.nnu, U.nnt, lane) : 0;
+  const int n_units = n_uneven > 0 ? n_uneven : U.total;
   int item = blockIdx.x / (NT * U.nnu), rem = blockIdx.x - item * (NT * U.nnu);
   const int step_item = gridDim.x / (NT * U.nnu), step_rem = gridDim.x - step_item * (NT * U.nnu);
-  for (int u = blockIdx.x; u < U.total; u += gridDim.x) {
-    const int ti = rem / U.nnu, nr = rem - ti * U.nnu;
-    const int cur_item = item;
-    item += step_item;
-    rem += step_rem;
-    if (rem >= NT * U.nnu) {
-      rem -= NT * U.nnu;
-      ++item;
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    int ti, cur_item, e0, e1;
+    if (n_uneven > 0) {
+      // the item whose units hold u: the last t with NT * c_pref[t] <= u
+      int lo_t = 0, hi_t = n_items - 1;
+      while (lo_t < hi_t) {
+        const int mid = (lo_t + hi_t + 1) >> 1;
+        if (NT * S.c_pref[mid] <= u) lo_t = mid;
+        else hi_t = mid - 1;
+      }
+      cur_item = lo_t;
+      const int k = S.c_pref[lo_t + 1] - S.c_pref[lo_t];
+      const int local = u - NT * S.c_pref[lo_t];
+      ti = local / k;
+      const int j = local - ti * k;
+      e0 = j * U.nnt / k;
+      e1 = (j + 1) * U.nnt / k;
+    } else {
+      ti = rem / U.nnu;
+      const int nr = rem - ti * U.nnu;
+      cur_item = item;
+      item += step_item;
+      rem += step_rem;
+      if (rem >= NT * U.nnu) {
+        rem -= NT * U.nnu;
+        ++item;
+      }
+      e0 = nr * U.npu;
+      e1 = MODE == kShrinkOnly ? e0 : min(e0 + U.npu, U.nnt);
     }
     // ---- the item and its slot on target ti
     int4 d;
@@ -922,7 +981,6 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
     if (lane < kItemRows) R.rows[lane] = myrow;
     // ---- its tiles: the whole shrink, then the expand of column range nr
     const int ks = MODE == kExpandOnly ? U.nkt : 0;
-    const int e0 = nr * U.npu, e1 = MODE == kShrinkOnly ? e0 : min(e0 + U.npu, U.nnt);
     const int nvi = a.d_in / 8, nvo = a.d_out / 8;
     for (int t = ks; t < U.nkt + (e1 - e0); ++t) {
       const bool shrink = t < U.nkt;
@@ -1294,6 +1352,7 @@ int launch_decode(lora_pool *pool, const DecodeCall &c, cudaStream_t st) {
   a.moe_e = c.moe_e;
   a.v = c.v;
   a.ldv = c.ldv;
+  a.n_sms = pool->decode_max_ctas / std::max(pool->decode_per_sm, 1);
   a.stall = c.stall;
   a.status = pool->d_status;
   a.wait_ns = g_wait_ns.load();
