@@ -83,6 +83,7 @@ _sig("lora_plan_layout_get", _I, [_P, _I, ctypes.POINTER(lora_plan_layout)])
 _sig("lora_plan_ids", _I, [_P, _P, _I, _P, _Z, _P])
 _sig("lora_plan_segments", _I, [_P, _P, _P, _I, _I, _P, _Z, _P])
 _sig("lora_mma_min_rows", _I, [])
+_sig("lora_mma_min_rows_for", _I, [_I, _I])
 _sig("lora_apply_plan", _I, [_P, _I, _P, _I, _P, _I, _P, _I, _P, _Z, _P])
 _sig("lora_apply", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _Z, _P])
 _sig("lora_apply_segments", _I, [_P, _I, _P, _I, _P, _I, _P, _P, _I, _P, _I, _P, _Z, _P])
@@ -251,6 +252,11 @@ def lora_plan_layout_get(pool: PoolHandle, T: int) -> lora_plan_layout:
 
 def lora_mma_min_rows() -> int:
     return int(_lib.lora_mma_min_rows())
+
+
+def lora_mma_min_rows_for(n_segments: int, T: int) -> int:
+    """Segment length from which a segment plan of this batch uses the tensor cores."""
+    return int(_lib.lora_mma_min_rows_for(n_segments, T))
 
 
 def lora_plan_ids(pool: PoolHandle, ids, ws, stream=None) -> None:

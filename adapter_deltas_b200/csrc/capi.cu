@@ -50,7 +50,9 @@ int check_linear(const lora_pool *p, int target, const void *x, int ldx, const v
   return LORA_OK;
 }
 
-enum { kPlanUnknown = 0, kPlanIds = 1, kPlanSegments = 2 };
+// kPlanSegmentsTiles: a segment plan that sent every segment to the
+// tensor-core tiles (segment_mma_min == 1): no short-segment decode items.
+enum { kPlanUnknown = 0, kPlanIds = 1, kPlanSegments = 2, kPlanSegmentsTiles = 3 };
 
 void set_plan_kind(lora_pool *p, const void *ws, int kind) {
   std::lock_guard<std::mutex> lk(p->mu);
@@ -92,6 +94,11 @@ int lora_plan_layout_get(const lora_pool *p, int T, lora_plan_layout *out) {
 
 int lora_mma_min_rows(void) { return kMmaMinRows; }
 
+int lora_mma_min_rows_for(int S, int T) {
+  if (S < 0 || T < 0 || T > kMaxTokens) return -1;
+  return segment_mma_min(S, T);
+}
+
 void lora_set_wait_limit_ns(uint64_t ns) { set_wait_limit_ns(ns); }
 
 int lora_plan_ids(lora_pool *p, const int32_t *ids, int T, void *ws, size_t ws_bytes, void *stream) {
@@ -113,7 +120,7 @@ int lora_plan_segments(lora_pool *p, const int32_t *seg_offsets, const int32_t *
   if (S > 0 && (!seg_offsets || !seg_slot)) return LORA_ERR_INVALID_ARG;
   DeviceGuard g(p->device);
   rc = launch_plan_segments(p, seg_offsets, seg_slot, S, T, ws, static_cast<cudaStream_t>(stream));
-  if (rc == LORA_OK) set_plan_kind(p, ws, kPlanSegments);
+  if (rc == LORA_OK) set_plan_kind(p, ws, segment_mma_min(S, T) == 1 ? kPlanSegmentsTiles : kPlanSegments);
   return rc;
 }
 
@@ -140,6 +147,8 @@ int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, i
   if (kind == kPlanIds)  // index-vector plans hold decode items only
     return launch_decode(p, c, st);
   PrefillGeometry geo;
+  if (kind == kPlanSegmentsTiles && prefill_geometry(p, target, plan_layout(T).j_max, &geo))
+    return launch_prefill(p, target, x, ldx, y, ldy, scales, T, ws, ws_bytes, st);  // every segment
   if (kind == kPlanSegments && prefill_geometry(p, target, plan_layout(T).j_max, &geo)) {
     // short segments on the decode kernel, long ones on the tensor cores
     rc = launch_decode(p, c, st);

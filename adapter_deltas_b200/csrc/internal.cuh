@@ -116,6 +116,14 @@ struct PlanLayout {
 
 constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Segment length from which a segment plan uses the tensor cores: a batch of
+// few segments (a prefill batch) sends every segment there, so that it needs
+// no decode launch for its short segments (a segment of m rows is one tile
+// of m rows: its adapter slices and rows are the same bytes either way);
+// otherwise segments of kMmaMinRows rows or more.  The few-segment rule
+// applies while the tiles stay within the plan's tile capacity.
+constexpr int kFewSegments = 16;
+
 constexpr PlanLayout plan_layout(int T) {
   PlanLayout L{};
   const int t = T > 0 ? T : 1;
@@ -132,6 +140,10 @@ constexpr PlanLayout plan_layout(int T) {
   L.tiles = off;     off = align256(off + size_t(L.j_max) * 16);
   L.total = off;
   return L;
+}
+
+constexpr int segment_mma_min(int S, int T) {
+  return (S <= kFewSegments && T / kMmaRows + S <= plan_layout(T).j_max) ? 1 : kMmaMinRows;
 }
 
 // Header words of a plan.

@@ -313,7 +313,7 @@ int launch_plan_segments(lora_pool *pool, const int32_t *off, const int32_t *slo
                          cudaStream_t st) {
   PlanLayout L = plan_layout(T);
   g_launches.fetch_add(1);
-  plan_segments_kernel<<<1, kPlanThreads, 0, st>>>(off, slot, S, T, kMmaMinRows, pool->view(), plan_view(ws, L),
+  plan_segments_kernel<<<1, kPlanThreads, 0, st>>>(off, slot, S, T, segment_mma_min(S, T), pool->view(), plan_view(ws, L),
                                                    pool->d_status);
   return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }

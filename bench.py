@@ -438,7 +438,10 @@ def run_b200(args, rank: int, world: int, local_rank: int):
     value = job_value(w.T, world, ms)
     if segmented:
         kernel_name = "prefill_kernels"
-        kernel_desc = "prefill_kernel (tcgen05) + decode_kernel launch for segments under %d rows" % L.lora_mma_min_rows()
+        kernel_desc = ("prefill kernels (tcgen05 shrink + expand) for every segment (%d segments)" % len(w.seg_slot)
+                       if L.lora_mma_min_rows_for(len(w.seg_slot), w.T) == 1 else
+                       "prefill kernels (tcgen05) + decode_kernel launch for segments under %d rows"
+                       % L.lora_mma_min_rows())
     elif one_launch:
         kernel_name, kernel_desc = "decode_kernel", "decode_kernel<fused> grouping the batch in-kernel (the whole step)"
     else:

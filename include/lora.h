@@ -270,9 +270,9 @@ LORA_API int lora_plan_ids(lora_pool *pool, const int32_t *ids, int T, void *ws,
  * seg_offsets[s] .. seg_offsets[s+1]-1 use slot seg_slot[s].
  *   seg_offsets  device int32 [S+1], non-decreasing, within [0, T];
  *   seg_slot     device int32 [S]; -1 = the segment has no adapter.
- * Segments at least lora_mma_min_rows() long take the tensor-core path (in
- * 128-row tiles) when the target allows it (r_max <= 32 and the slices fit in
- * shared memory), the others the decode path.  Offsets that decrease or leave
+ * Segments at least lora_mma_min_rows_for(S, T) long take the tensor-core
+ * path (in 128-row tiles) when the target allows it (r_max <= 32 and the
+ * slices fit in shared memory), the others the decode path.  Offsets that decrease or leave
  * [0, T] make the whole plan empty (LORA_ERR_BAD_ID); segments naming an
  * invalid slot are skipped (LORA_ERR_BAD_ID / LORA_ERR_NOT_LOADED).
  */
@@ -280,8 +280,20 @@ LORA_API int lora_plan_segments(lora_pool *pool, const int32_t *seg_offsets,
                        const int32_t *seg_slot, int S, int T, void *ws,
                        size_t ws_bytes, void *stream);
 
-/* Segment length from which the tensor-core path is used. */
+/* Segment length from which the tensor-core path is used in a batch of many
+ * segments. */
 LORA_API int lora_mma_min_rows(void);
+
+/*
+ * Segment length from which lora_plan_segments sends a segment to the
+ * tensor-core path, for a batch of S segments over T rows: 1 (every segment)
+ * when S <= 16 and the tiles fit the plan (floor(T / 128) + S tiles at most),
+ * so that a prefill batch needs no decode launch for its short segments (a
+ * segment of m rows is then one tile of m rows: the same adapter slices and
+ * rows as on the decode path); lora_mma_min_rows() otherwise.  -1 for S < 0
+ * or T outside [0, 2^20].
+ */
+LORA_API int lora_mma_min_rows_for(int S, int T);
 
 /*
  * Apply a built plan to one target:  y[t] += scales[a] * B_a (A_a x[t]).

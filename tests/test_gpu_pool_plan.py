@@ -89,7 +89,7 @@ def test_plan_segments_bit_exact(cuda_device):
         assert np.array_equal(perm, np.arange(w.T))
         assert np.array_equal(seg_start, w.seg_offsets)
         assert np.array_equal(seg_slot, w.seg_slot)
-        mma = L.lora_mma_min_rows()
+        mma = L.lora_mma_min_rows_for(len(w.seg_slot), w.T)
         covered = []
         for slot, r0, m, seg in tiles.tolist():
             assert seg_slot[seg] == slot and seg_start[seg + 1] - seg_start[seg] >= mma

@@ -1,6 +1,7 @@
-"""GPU parity of the segment (prefill) path: long segments on the tensor cores
+"""GPU parity of the segment (prefill) path: segments on the tensor cores
 (tcgen05 MMA, TMA tiles; 128-row tiles, a shrink launch over k-slices and an
-expand launch over column groups), short segments on the decode kernel,
+expand launch over column groups) -- every segment of a batch of at most 16,
+else those of 64 rows or more, the short ones then on the decode kernel --
 against the fp64 oracle on the same seeded inputs.
 
 Bound: max |y_gpu - y_ref| <= 4e-3 * max |y_ref|, with the base output and
@@ -79,12 +80,34 @@ def test_prefill_config_uses_tensor_cores_and_matches(cuda_device):
     with DevicePool(w, cuda_device) as pool:
         n0 = L.lora_kernel_launches()
         got = _run_segments(pool, w, 0, w.x(0), w.y_in(0), w.seg_offsets, w.seg_slot)
-        assert L.lora_kernel_launches() - n0 == 4  # plan, decode (short segments), tensor-core shrink, expand
+        # 8 segments: every one on the tensor cores, no short-segment decode launch
+        assert L.lora_mma_min_rows_for(len(w.seg_slot), w.T) == 1
+        assert L.lora_kernel_launches() - n0 == 3  # plan, tensor-core shrink, expand
         ref, _ = oracle_y(w, 0, w.x(0), w.y_in(0), w.ids)
         assert_close(got, ref, what="config 3")
         got0 = _run_segments(pool, w, 0, w.x(0), np.zeros_like(w.y_in(0)), w.seg_offsets, w.seg_slot)
         ref0, _ = oracle_y(w, 0, w.x(0), np.zeros_like(w.y_in(0)), w.ids)
         assert_close(got0, ref0, what="config 3 delta only")
+
+
+def test_many_segments_split_between_tensor_cores_and_decode(cuda_device):
+    # 24 segments: those of 64 rows or more on the tensor cores, the short
+    # ones (1 - 63 rows) on the decode kernel, in one apply of four launches
+    lengths = [300, 5, 1, 63, 64, 70, 2, 3, 129, 17, 40, 1, 128, 9, 33, 200, 6, 7, 64, 11, 1, 90, 12, 2]
+    slots = [i % 5 for i in range(len(lengths))]
+    off, seg_slot = _segments(lengths, slots, gap_rows=(4,))
+    T = int(off[-1])
+    assert L.lora_mma_min_rows_for(len(seg_slot), T) == L.lora_mma_min_rows() == 64
+    w = _make(T, 512, 384, [16, 8, 16, 13, 16], 16, seed=5)
+    ids = _ids(off, seg_slot)
+    with DevicePool(w, cuda_device) as pool:
+        n0 = L.lora_kernel_launches()
+        got = _run_segments(pool, w, 0, w.x(0), w.y_in(0), off, seg_slot)
+        assert L.lora_kernel_launches() - n0 == 4  # plan, decode (short segments), tensor-core shrink, expand
+        ref, _ = oracle_y(w, 0, w.x(0), w.y_in(0), ids)
+        assert_close(got, ref, what="24 segments")
+        none = ids < 0
+        assert np.array_equal(got[none], w.y_in(0)[none])
 
 
 def test_rank_32_and_distinct_scales(cuda_device):
