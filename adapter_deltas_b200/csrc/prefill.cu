@@ -97,13 +97,13 @@ __device__ __forceinline__ const uint8_t *block_chunk(const PoolView &pool, int 
 // ============================================================ shrink kernel
 struct ShSmem {
   uint8_t *ring, *aw, *stg;  // x stages; A slice in the MMA layout; A slice rows as copied
-  uint64_t *full, *empty, *w_full, *a_land, *sh_done;
+  uint64_t *full, *empty, *w_full, *a_land, *sh_done, *stg_free;
   uint32_t *tmem_slot;
 };
 
 __host__ __device__ inline int sh_smem_bytes(int n_stages, int r_cap, int kb_per) {
   return 1024 /* alignment slack */ + n_stages * kBoxBytes + 2 * r_cap * kb_per * kBoxCols * 2 +
-         (2 * kShMaxStages + 3) * 8 + 16;
+         (2 * kShMaxStages + 4) * 8 + 16;
 }
 
 // Warp roles: warps 0-3 copy the adapter slice and write the partial V (warp
@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     S.w_full = b++;
     S.a_land = b++;
     S.sh_done = b++;
+    S.stg_free = b++;
     S.tmem_slot = reinterpret_cast<uint32_t *>(b);
   }
   if (warp == 0) {
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     mbar_init(S.w_full, kShEpiThreads);
     mbar_init(S.a_land, 1);
     mbar_init(S.sh_done, 1);
+    mbar_init(S.stg_free, 1);
     fence_mbar_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&a.tmap_x)) : "memory");
   }
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
   const uint32_t aw_u = smem_u32(S.aw), ring_u = smem_u32(S.ring);
   uint32_t gbase = 0;   // ring uses so far: use g sits in stage g % NS with phase (g / NS) & 1
   uint32_t ucount = 0;  // units multiplied so far (w_full / sh_done phases)
-  uint32_t ucopy = 0;   // units whose A slice was copied (a_land phases)
+  uint32_t ucopy = 0;   // units whose A slice was copied (a_land phases; stg_free phases: ucopy - 1)
 
   for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
     const int tile = u / a.n_ks, ks = u - tile * a.n_ks;
@@ -168,23 +170,6 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     const int4 d = a.tiles[tile];
     const int slot = d.x, row0 = d.y, m = d.z;
 
-    if (warp == kShEpiWarps) {
-      // ------------------------------------------------ TMA producer
-      // (x depends only on the tile record: the stream starts at once; a
-      // unit whose adapter turns out absent still passes its blocks through
-      // the ring, the MMA warp just does not multiply them)
-      if (lane == 0) {
-        for (int i = 0; i < nkb; ++i) {
-          const uint32_t g = gbase + i, st = g % NS;
-          if (g >= (uint32_t)NS && !pf_wait(&S.empty[st], ((g / NS) - 1) & 1, a.status, alive)) break;
-          mbar_arrive_expect_tx(&S.full[st], kBoxBytes);
-          tma_load_2d(S.ring + st * kBoxBytes, &a.tmap_x, (kb0 + i) * kBoxCols, row0, &S.full[st]);
-        }
-      }
-      __syncwarp();
-      gbase += nkb;
-      continue;
-    }
     // The A slice does not wait for the rank: all r_cap rows come (the pool
     // keeps an adapter's rows past its rank at zero), so the copies leave as
     // soon as the tile record is known.
@@ -195,15 +180,37 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     const int tc = pool_tile_cols(a.pool_r_max), tcc = tc / 8;
     const int tile0 = kb0 * kBoxCols / tc, n_tl = (cols + tc - 1) / tc;
     const int rows_cp = min(a.r_cap, a.pool_r_max);
-    if (warp == 0) {
+
+    if (warp == kShEpiWarps) {
+      // ------------------------------------------------ TMA producer
+      // The A slice first (the MMAs wait for it; issued behind this CTA's
+      // x boxes it would queue behind every CTA's first wave of x), once the
+      // epilogue is done with the previous unit's staged slice; then the x
+      // boxes (x depends only on the tile record; a unit whose adapter turns
+      // out absent still passes its blocks through the ring, the MMA warp
+      // just does not multiply them).
+      if (ucopy > 0) warp_wait(S.stg_free, (ucopy - 1) & 1u, a.status, alive);
       if (lane == 0) mbar_arrive_expect_tx(S.a_land, (uint32_t)rows_cp * (uint32_t)cols * 2u);
       __syncwarp();
-      if (lane < n_tl) {
+      if (lane < n_tl && alive) {
         const int t = tile0 + lane;
         const int tw = min(tcc, a.d_in / 8 - t * tcc);
         copy_pool_row(a.pool, slot, a.a_off + (long long)t * a.pool_r_max * tcc * 16, (uint32_t)(rows_cp * tw * 16),
                       S.stg + lane * a.r_cap * tcc * 16, S.a_land, a.status);
       }
+      __syncwarp();
+      if (lane == 0) {
+        for (int i = 0; i < nkb; ++i) {
+          const uint32_t g = gbase + i, st = g % NS;
+          if (g >= (uint32_t)NS && !pf_wait(&S.empty[st], ((g / NS) - 1) & 1, a.status, alive)) break;
+          mbar_arrive_expect_tx(&S.full[st], kBoxBytes);
+          tma_load_2d(S.ring + st * kBoxBytes, &a.tmap_x, (kb0 + i) * kBoxCols, row0, &S.full[st]);
+        }
+      }
+      __syncwarp();
+      gbase += nkb;
+      ++ucopy;
+      continue;
     }
     const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
     const bool use = r > 0 && r <= a.r_cap;
@@ -244,12 +251,13 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
       if (use) {
         const int kv_n = nkb * (kBoxCols / 8);
         const int jl = lane & 7, vo = lane >> 3;
+        const int tsh = 31 - __clz(tcc);  // (tcc is a power of two)
         for (int jg = 0; jg < R / 8; ++jg) {
           const int j = jg * 8 + jl;
           for (int kv = warp * 4 + vo; kv < kv_n; kv += kShEpiWarps * 4) {
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (j < r && kv * 8 < cols) {
-              const int tl = kv / tcc, c = kv - tl * tcc;
+              const int tl = kv >> tsh, c = kv & (tcc - 1);
               const int tw = min(tcc, a.d_in / 8 - (tile0 + tl) * tcc);
               v = *reinterpret_cast<const uint4 *>(S.stg + (tl * a.r_cap * tcc + j * tw + swz_chunk(c, j, tw)) * 16);
             }
@@ -283,6 +291,7 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     // the epilogue warps stay in step (an absent adapter's unit has no
     // other barrier that would hold them together)
     if (warp < kShEpiWarps) asm volatile("bar.sync 1, %0;" ::"n"(kShEpiThreads) : "memory");
+    if (tid == 0) pf_arrive(S.stg_free);  // the staged slice may be overwritten
     gbase += nkb;
     if (use) ++ucount;
     ++ucopy;
