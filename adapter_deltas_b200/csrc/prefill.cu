@@ -366,6 +366,7 @@ __global__ void __launch_bounds__(kExThreads, kExMaxPerSm) pf_expand_kernel(cons
     const int4 d = a.tiles[tile];
     const int slot = d.x, row0 = d.y, m = d.z;
     const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
+    const float scale = a.scales[slot];  // (read here: its latency overlaps the unit's loads)
     if (r <= 0 || r > a.r_cap) continue;  // reported by the shrink kernel
     const int R = (r + 15) & ~15;
     const uint32_t par = ucount & 1u;
@@ -470,7 +471,6 @@ __global__ void __launch_bounds__(kExThreads, kExMaxPerSm) pf_expand_kernel(cons
       tmem_wait_ld();
       uint8_t *box = S.ys + b * kBoxBytes;
       const int row = lg * 32 + lane;
-      const float scale = a.scales[slot];
       uint4 yv[8];
 #pragma unroll
       for (int c16 = 0; c16 < 8; ++c16) yv[c16] = *reinterpret_cast<const uint4 *>(box + row * 128 + ((c16 ^ (row & 7)) * 16));
