@@ -516,8 +516,7 @@ LORA_API int lora_expand(lora_pool *pool, int target, const float *v, int ldv, v
  *   - T > LORA_NOALLOC_MAX_TOKENS returns LORA_ERR_WORKSPACE (nothing runs).
  *   - The first call on a device looks up the array's device address (a
  *     runtime query, done with that device current, and again after a device
- *     reset or from another driver context); make that first call before
- *     capturing a stream into a CUDA graph.
+ *     reset or from another driver context).
  *   - All calls of more than 256 rows share the one array, which keeps the
  *     last call's plan.  No part of it needs clearing (each call rewrites
  *     everything it reads), but such calls that overlap on the GPU -- on
