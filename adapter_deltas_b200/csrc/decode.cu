@@ -25,13 +25,19 @@
 // synchronisation, no scratch memory, and every row's v is summed in the same
 // fixed order whatever the batch, the path or the launch.
 //
+// Column ranges per item: enough for about one unit per CTA, uniform over the
+// items; when that still leaves SMs idle, items of many rows (whose expand
+// tiles carry many y rows) get twice as many (uneven_ranges).
+//
 // B200 mapping.  Per CTA one producer warp walks the CTA's units and streams
 // their tiles into a shared-memory ring with 1-D bulk async copies
 // (cp.async.bulk, no multicast): the first r rows of an adapter tile are one
 // contiguous range of the pool's tiled block (one copy), activation rows one
 // copy each; the copies complete on mbarriers.  Eight consumer warps run the
-// contractions on warp-level bf16 MMA and write y.  The producer runs up to
-// the ring depth ahead of them.
+// contractions on warp-level bf16 MMA (a full tile on a compile-time
+// schedule), update the staged y rows in place with ldmatrix / stmatrix and
+// send them out -- coalesced stores for small items, one bulk copy per row
+// for larger ones.  The producer runs up to the ring depth ahead of them.
 #include <algorithm>
 #include <climits>
 
