@@ -57,7 +57,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         objs.append(obj)
     tmp = LIB + ".tmp.%d" % os.getpid()
     subprocess.run([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
-                    "-o", tmp, *objs], check=True)
+                    "-o", tmp, *objs, "-ldl"], check=True)
     os.replace(tmp, LIB)
     return LIB
 

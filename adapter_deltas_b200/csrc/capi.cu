@@ -102,6 +102,7 @@ int lora_mma_min_rows_for(int S, int T) {
 void lora_set_wait_limit_ns(uint64_t ns) { set_wait_limit_ns(ns); }
 
 int lora_plan_ids(lora_pool *p, const int32_t *ids, int T, void *ws, size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_plan_ids");
   int rc = check_call(p, 0, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
   if (!ids) return LORA_ERR_INVALID_ARG;
@@ -113,6 +114,7 @@ int lora_plan_ids(lora_pool *p, const int32_t *ids, int T, void *ws, size_t ws_b
 
 int lora_plan_segments(lora_pool *p, const int32_t *seg_offsets, const int32_t *seg_slot, int S, int T, void *ws,
                        size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_plan_segments");
   int rc = check_call(p, 0, T, ws, ws_bytes);
   if (rc != LORA_OK) return rc;
   if (S < 0 || S > kMaxTokens) return LORA_ERR_INVALID_ARG;
@@ -126,6 +128,7 @@ int lora_plan_segments(lora_pool *p, const int32_t *seg_offsets, const int32_t *
 
 int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const float *scales, int T,
                     const void *ws, size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_apply_plan");
   int rc = check_call(p, target, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
   if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
@@ -162,6 +165,7 @@ int lora_apply_plan(lora_pool *p, int target, const void *x, int ldx, void *y, i
 
 int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const int32_t *ids,
                const float *scales, int T, void *ws, size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_apply");
   int rc = check_call(p, target, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
   if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
@@ -188,6 +192,7 @@ int lora_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ld
 
 int lora_selftest_stalled_apply(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
                                 const int32_t *ids, const float *scales, int T, void *stream) {
+  NvtxRange nvtx_range("lora_selftest_stalled_apply");
   if (!p || target < 0 || target >= p->n_targets || T < 0 || T > kFusedMaxT) return LORA_ERR_INVALID_ARG;
   if (T == 0) return LORA_OK;
   int rc;
@@ -212,6 +217,7 @@ int lora_selftest_stalled_apply(lora_pool *p, int target, const void *x, int ldx
 int lora_apply_multi(lora_pool *p, int n_targets, const int *targets, const void *x, int ldx, void *y, int ldy,
                      const int *y_cols, const int32_t *ids, const float *scales, int T, void *ws, size_t ws_bytes,
                      void *stream) {
+  NvtxRange nvtx_range("lora_apply_multi");
   if (!p || !targets || !y_cols || n_targets < 1 || n_targets > kMaxMulti) return LORA_ERR_INVALID_ARG;
   int rc = check_call(p, targets[0], T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
@@ -254,6 +260,7 @@ int lora_apply_multi(lora_pool *p, int n_targets, const int *targets, const void
 int lora_apply_segments(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
                         const int32_t *seg_offsets, const int32_t *seg_slot, int S, const float *scales, int T,
                         void *ws, size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_apply_segments");
   int rc = check_call(p, target, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
   if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
@@ -266,6 +273,7 @@ int lora_apply_segments(lora_pool *p, int target, const void *x, int ldx, void *
 
 int lora_shrink(lora_pool *p, int target, const void *x, int ldx, const int32_t *ids, int T, float *v, int ldv,
                 void *ws, size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_shrink");
   int rc = check_call(p, target, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
   if ((rc = check_rows(x, ldx, p->targets[target].d_in)) != LORA_OK) return rc;
@@ -292,6 +300,7 @@ int lora_shrink(lora_pool *p, int target, const void *x, int ldx, const int32_t 
 
 int lora_expand(lora_pool *p, int target, const float *v, int ldv, void *y, int ldy, const int32_t *ids,
                 const float *scales, int T, void *ws, size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_expand");
   int rc = check_call(p, target, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
   if ((rc = check_rows(y, ldy, p->targets[target].d_out)) != LORA_OK) return rc;
@@ -324,6 +333,7 @@ size_t lora_linear_workspace_bytes(const lora_pool *p, int target, int max_token
 
 int lora_linear(lora_pool *p, int target, const void *x, int ldx, const void *W, int ldw, void *y, int ldy,
                 const int32_t *ids, const float *scales, int T, void *ws, size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_linear");
   int rc = check_call(p, target, T, ws, ws_bytes);
   if (rc != LORA_OK || T == 0) return rc;
   if ((rc = check_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, T)) != LORA_OK) return rc;
@@ -338,6 +348,7 @@ int lora_linear(lora_pool *p, int target, const void *x, int ldx, const void *W,
 
 int lora_linear_expand(lora_pool *p, int target, const void *x, int ldx, const void *W, int ldw, const float *v,
                        int ldv, void *y, int ldy, const int32_t *ids, const float *scales, int T, void *stream) {
+  NvtxRange nvtx_range("lora_linear_expand");
   if (!p || target < 0 || target >= p->n_targets || T < 0 || T > kMaxTokens) return LORA_ERR_INVALID_ARG;
   if (T == 0) return LORA_OK;
   int rc = check_linear(p, target, x, ldx, W, ldw, y, ldy, ids, scales, T);
@@ -356,6 +367,7 @@ size_t lora_moe_workspace_bytes(const lora_pool *p, int target, int max_pairs) {
 int lora_apply_moe(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy, const int32_t *lora_ids,
                    const int32_t *topk_ids, int T, int top_k, int n_experts, const float *scales, void *ws,
                    size_t ws_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_apply_moe");
   if (!p || target < 0 || target >= p->n_targets || T < 0) return LORA_ERR_INVALID_ARG;
   if (top_k < 1 || n_experts < 1 || (long long)T * top_k > kMaxTokens) return LORA_ERR_INVALID_ARG;
   const int n_pairs = T * top_k;

@@ -15,9 +15,20 @@
 #include <unordered_map>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "lora.h"
 
 namespace lora {
+
+// A named NVTX range over one C-ABI call (host side: seen by profilers that
+// record NVTX ranges, a few nanoseconds otherwise).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // ---------------------------------------------------------------- limits
 constexpr int kRMax = 64;            // largest slot rank

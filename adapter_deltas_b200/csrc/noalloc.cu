@@ -76,6 +76,7 @@ using namespace lora;
 
 extern "C" int lora_apply_noalloc(lora_pool *p, int target, const void *x, int ldx, void *y, int ldy,
                                   const int32_t *ids, const float *scales, int T, void *stream) {
+  NvtxRange nvtx_range("lora_apply_noalloc");
   if (!p || target < 0 || target >= p->n_targets || T < 0) return LORA_ERR_INVALID_ARG;
   if (T == 0) return LORA_OK;
   if (T > LORA_NOALLOC_MAX_TOKENS || plan_layout(T).total > kNoAllocBytes) return LORA_ERR_WORKSPACE;

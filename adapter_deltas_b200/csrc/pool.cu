@@ -296,6 +296,7 @@ int lora_pool_create(lora_pool **out, int device, const lora_target *targets, in
 
 int lora_pool_load(lora_pool *p, int slot, int target, int rank, const void *A, const void *B,
                    int src_is_device, void *stream) {
+  NvtxRange nvtx_range("lora_pool_load");
   if (!p) return LORA_ERR_INVALID_ARG;
   if (slot < 0 || slot >= p->n_slots) return LORA_ERR_SLOT;
   if (target < 0 || target >= p->n_targets) return LORA_ERR_INVALID_ARG;
@@ -373,6 +374,7 @@ size_t lora_swap_staging_bytes(const lora_pool *p, const int *ranks) {
 
 int lora_pool_swap_in(lora_pool *p, int slot, const int *ranks, const void *src, size_t src_bytes, void *staging,
                       size_t staging_bytes, void *stream) {
+  NvtxRange nvtx_range("lora_pool_swap_in");
   if (!p || !ranks) return LORA_ERR_INVALID_ARG;
   if (slot < 0 || slot >= p->n_slots) return LORA_ERR_SLOT;
   const long long need = swap_src_bytes(p, ranks);
