@@ -18,12 +18,14 @@ import os
 from typing import Optional, Sequence, Tuple
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblora_b200.so")
+# LORA_B200_DEBUG=1 selects the bounds-checking build (LORA_DEBUG)
+DEBUG_BUILD = os.environ.get("LORA_B200_DEBUG") == "1"
+LIB_PATH = os.path.join(_HERE, "liblora_b200_debug.so" if DEBUG_BUILD else "liblora_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        "liblora_b200.so is not built; run `python adapter_deltas_b200/_build.py` "
-        "(the delta path has no fallback)")
+        "%s is not built; run `python adapter_deltas_b200/_build.py%s` "
+        "(the delta path has no fallback)" % (os.path.basename(LIB_PATH), " --debug" if DEBUG_BUILD else ""))
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -41,6 +43,7 @@ LORA_ERR_CUDA = 6
 LORA_ERR_BAD_ID = 7
 LORA_ERR_TIMEOUT = 8
 LORA_ERR_WORKSPACE = 9
+LORA_ERR_BOUNDS = 10
 
 
 class lora_target(ctypes.Structure):

@@ -800,6 +800,10 @@ __device__ int plan_cache(const DecodeArgs &a, const DecSmem &S, int tid) {
   const int n_items = min(a.hdr[a.items_hdr], a.items_cap);
   if (tid < n_ci && tid < n_items) {
     const PoolView &p = a.pool;
+    // (LORA_DEBUG: an item outside the pool's slots or the batch's rows is dropped)
+    if (!dbg_ok(d.x >= 0 && d.x < p.n_slots && d.y >= 0 && d.z >= 0 && d.z <= kItemRows && d.y + d.z <= a.T,
+                a.status))
+      d = make_int4(0, 0, 0, 0);
     const int slot = d.x;
     const int rk = p.rank[(long long)slot * p.n_targets + a.tgt[0]];
     const int pa = block_page(p, slot, a.a_off[0], (long long)a.r_max * a.d_in * 2);
@@ -947,6 +951,9 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
     int4 d;
     if (cur_item < n_cached) d = S.c_item[cur_item];
     else d = a.items[cur_item];
+    if (!dbg_ok(d.x >= 0 && d.x < a.pool.n_slots && d.y >= 0 && d.z >= 0 && d.z <= kItemRows && d.y + d.z <= a.T,
+                a.status))
+      d = make_int4(0, 0, 0, 0);  // (LORA_DEBUG: dropped)
     const int slot = d.x, first = d.y, m = d.z;
     int r, page_a, page_b;
     float scale;
@@ -969,9 +976,11 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
       scale = __int_as_float(__shfl_sync(0xffffffffu, val, 3));
     }
     if (r <= 0 || m <= 0) continue;  // nothing to add (a slot without this target)
-    const int myrow = lane < m ? (first + lane < perm_cached ? S.c_perm[first + lane] : a.perm[first + lane]) : 0;
+    int myrow = lane < m ? (first + lane < perm_cached ? S.c_perm[first + lane] : a.perm[first + lane]) : 0;
+    if (lane < m && !dbg_ok(myrow >= 0 && myrow < a.T, a.status)) myrow = -1;  // (LORA_DEBUG: not read or written)
     // lane L (1 <= L <= m) copies activation row L - 1: its x row and y row
-    const int arow = __shfl_sync(0xffffffffu, myrow, (lane + 31) & 31);
+    const int arow_raw = __shfl_sync(0xffffffffu, myrow, (lane + 31) & 31);
+    const int arow = kDebugChecks && arow_raw < 0 ? 0 : arow_raw;
     const uint8_t *x_row = reinterpret_cast<const uint8_t *>(a.x + (long long)(arow / a.x_div) * a.ldx);
     const long long a_blk = S.tg[ti], b_blk = S.tg[kMaxMulti + ti], ycol = S.tg[2 * kMaxMulti + ti];
     const uint8_t *y_row = reinterpret_cast<const uint8_t *>(a.y + (long long)arow * a.ldy + ycol);
@@ -1007,7 +1016,10 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
         const long long off = (shrink ? a_blk : b_blk) + tt * tile_stride;
         const int page = shrink ? page_a : page_b;
         const uint32_t bytes = (uint32_t)r * row_bytes;
-        if (page >= 0) bulk_g2s(buf, page_addr(a.pool, page, off), bytes, &S.full[stage]);
+        if (page >= 0) {
+          if (dbg_page_range(a.pool, page, off, bytes, a.status)) bulk_g2s(buf, page_addr(a.pool, page, off), bytes, &S.full[stage]);
+          else bulk_g2s_redirect(buf, a.pool, bytes, &S.full[stage]);
+        }
         else copy_pool_row(a.pool, slot, off, bytes, buf, &S.full[stage], a.status);
       }
       __syncwarp();  // (the expected bytes are registered before any copy can land)
@@ -1114,7 +1126,7 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) s += red[w * kItemRows * r + i * r + j];
               }
-              a.v[(long long)R.rows[i] * a.ldv + j] = s;
+              if (!kDebugChecks || R.rows[i] >= 0) a.v[(long long)R.rows[i] * a.ldv + j] = s;
             }
           } else {
             for (int e = tid; e < n; e += kConsumerThreads) {
@@ -1141,7 +1153,7 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
       if (MODE == kExpandOnly && first) {  // the caller's v
         for (int e = tid; e < m * r; e += kConsumerThreads) {
           const int i = e / r, j = e - i * r;
-          S.v[i * a.r_max + j] = a.v[(long long)R.rows[i] * a.ldv + j];
+          S.v[i * a.r_max + j] = (!kDebugChecks || R.rows[i] >= 0) ? a.v[(long long)R.rows[i] * a.ldv + j] : 0.f;
         }
       }
       cons_sync();  // S.v complete (written by the shrink's last tile or just above)
@@ -1156,6 +1168,7 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
       if (m <= kStoreRowsMax) {
         cons_sync();
         for (int i = warp; i < m; i += kConsumerWarps) {
+          if (kDebugChecks && R.rows[i] < 0) continue;  // (LORA_DEBUG: a row that failed its check)
           const uint8_t *src = yb + i * pitch;
           uint16_t *dst = a.y + (long long)R.rows[i] * a.ldy + R.ycol + (long long)v_lo * 8;
           for (int ch = lane; ch < wv; ch += 32)
@@ -1167,8 +1180,9 @@ __device__ void consume(const DecodeArgs &a, const DecSmem &S, int tid) {
         cons_sync();
         if (lane == 0) {
           const long long col = R.ycol + (long long)v_lo * 8;
-          if (warp < m) bulk_s2g(a.y + (long long)R.rows[warp] * a.ldy + col, yb + warp * pitch, (uint32_t)wv * 16u);
-          if (warp + 8 < m)
+          if (warp < m && (!kDebugChecks || R.rows[warp] >= 0))
+            bulk_s2g(a.y + (long long)R.rows[warp] * a.ldy + col, yb + warp * pitch, (uint32_t)wv * 16u);
+          if (warp + 8 < m && (!kDebugChecks || R.rows[warp + 8] >= 0))
             bulk_s2g(a.y + (long long)R.rows[warp + 8] * a.ldy + col, yb + (warp + 8) * pitch, (uint32_t)wv * 16u);
           bulk_commit();
         }

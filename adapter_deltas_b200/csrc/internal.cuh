@@ -59,7 +59,31 @@ struct PoolView {
   int log2_page;           // -1: one page per slot
   int n_slots;
   int n_targets;
+  int n_pages;             // physical pages of the pool memory
 };
+
+// LORA_DEBUG builds check each index, page and byte range before it is used
+// for a load, a copy or a store; dbg_ok() records LORA_ERR_BOUNDS in the
+// sticky status and returns false where a check fails (the caller then skips
+// or redirects the access).  Other builds compile the checks away.
+#ifdef LORA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool dbg_ok(bool ok, int *status) {
+  if (!kDebugChecks) return true;
+  if (!ok) atomicCAS(status, 0, LORA_ERR_BOUNDS);
+  return ok;
+}
+// LORA_DEBUG: the slot range [off, off + bytes) of a slot lies inside the
+// slot, and each page it touches inside the pool memory.
+__device__ __forceinline__ bool dbg_slot_range(const PoolView &p, int slot, long long off, long long bytes,
+                                               int *status) {
+  if (!kDebugChecks) return true;
+  const long long slot_bytes = p.log2_page < 0 ? p.page_bytes : (long long)p.pps * p.page_bytes;
+  return dbg_ok(slot >= 0 && slot < p.n_slots && off >= 0 && bytes >= 0 && off + bytes <= slot_bytes, status);
+}
 
 // Physical address of logical byte `off` of `slot`, and how many bytes stay
 // on the same page from there.
@@ -320,11 +344,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ void set_status(int *status, int code) { atomicCAS(status, 0, code); }
 
+// LORA_DEBUG: `bytes` from the pool's first page(s) instead of a range that
+// failed its check, so that the bytes a stage expects still arrive.
+__device__ __forceinline__ void bulk_g2s_redirect(uint8_t *dst, const PoolView &pool, uint32_t bytes,
+                                                  uint64_t *bar) {
+  while (bytes > 0) {
+    const uint32_t n = (uint32_t)min((long long)bytes, pool.page_bytes);
+    bulk_g2s(dst, pool.base, n, bar);
+    dst += n;
+    bytes -= n;
+  }
+}
+// LORA_DEBUG: `bytes` from logical byte `off` of a block on physical page
+// `page` stay inside that page and the page inside the pool memory.
+__device__ __forceinline__ bool dbg_page_range(const PoolView &p, int page, long long off, long long bytes,
+                                               int *status) {
+  if (!kDebugChecks) return true;
+  const long long inside = p.log2_page < 0 ? off : (off & (p.page_bytes - 1));
+  return dbg_ok(page >= 0 && page < p.n_pages && inside >= 0 && inside + bytes <= p.page_bytes, status);
+}
+
 // Copy `bytes` of slot's logical range starting at `off` into dst, cut at
 // page boundaries.  A missing page (slot unloaded under our feet) is replaced
 // by page-free reads of the pool base and reported.
 __device__ __forceinline__ void copy_pool_row(const PoolView &pool, int slot, long long off, uint32_t bytes,
                                               uint8_t *dst, uint64_t *bar, int *status) {
+  if (!dbg_slot_range(pool, slot, off, bytes, status)) {
+    bulk_g2s_redirect(dst, pool, bytes, bar);
+    return;
+  }
   while (bytes > 0) {
     long long room;
     const uint8_t *src = pool_addr(pool, slot, off, &room);
@@ -333,6 +381,9 @@ __device__ __forceinline__ void copy_pool_row(const PoolView &pool, int slot, lo
       set_status(status, LORA_ERR_NOT_LOADED);
       src = pool.base;
     }
+    if (kDebugChecks && src != pool.base &&
+        !dbg_ok(src >= pool.base && src + n <= pool.base + (long long)pool.n_pages * pool.page_bytes, status))
+      src = pool.base;
     bulk_g2s(dst, src, n, bar);
     dst += n;
     off += n;
@@ -393,6 +444,7 @@ struct lora_pool {
     v.log2_page = log2_page;
     v.n_slots = n_slots;
     v.n_targets = n_targets;
+    v.n_pages = n_pages;
     return v;
   }
 };

@@ -197,6 +197,7 @@ const char *lora_status_string(int s) {
     case LORA_ERR_BAD_ID: return "LORA_ERR_BAD_ID";
     case LORA_ERR_TIMEOUT: return "LORA_ERR_TIMEOUT";
     case LORA_ERR_WORKSPACE: return "LORA_ERR_WORKSPACE";
+    case LORA_ERR_BOUNDS: return "LORA_ERR_BOUNDS";
     default: return "LORA_ERR_UNKNOWN";
   }
 }

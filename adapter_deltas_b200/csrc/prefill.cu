@@ -84,7 +84,8 @@ struct __align__(64) PrefillArgs {
 // the block's page when it has one (page >= 0), else through the page table.
 __device__ __forceinline__ const uint8_t *block_chunk(const PoolView &pool, int slot, int page, long long off,
                                                       int *status) {
-  if (page >= 0) return page_addr(pool, page, off);
+  if (page >= 0) return dbg_page_range(pool, page, off, 16, status) ? page_addr(pool, page, off) : pool.base;
+  if (!dbg_slot_range(pool, slot, off, 16, status)) return pool.base;  // (LORA_DEBUG: redirected)
   long long room;
   const uint8_t *src = pool_addr(pool, slot, off, &room);
   if (!src) {
@@ -168,6 +169,10 @@ __global__ void __launch_bounds__(kShThreads, 1) pf_shrink_kernel(const __grid_c
     const int kb0 = ks * a.kb_per, nkb = min(a.kb_per, nkb_all - kb0);
     if (nkb <= 0) continue;
     const int4 d = a.tiles[tile];
+    // (LORA_DEBUG: a tile outside the pool's slots or the batch's rows is skipped by every role)
+    if (!dbg_ok(d.x >= 0 && d.x < a.pool.n_slots && d.y >= 0 && d.z > 0 && d.z <= kMmaRows && d.y + d.z <= a.T,
+                a.status))
+      continue;
     const int slot = d.x, row0 = d.y, m = d.z;
 
     // The A slice does not wait for the rank: all r_cap rows come (the pool
@@ -364,6 +369,10 @@ __global__ void __launch_bounds__(kExThreads, kExMaxPerSm) pf_expand_kernel(cons
   for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
     const int tile = u / a.n_groups, grp = u - tile * a.n_groups;
     const int4 d = a.tiles[tile];
+    // (LORA_DEBUG: a tile outside the pool's slots or the batch's rows is skipped by every role)
+    if (!dbg_ok(d.x >= 0 && d.x < a.pool.n_slots && d.y >= 0 && d.z > 0 && d.z <= kMmaRows && d.y + d.z <= a.T,
+                a.status))
+      continue;
     const int slot = d.x, row0 = d.y, m = d.z;
     const int r = a.pool.rank[slot * a.pool.n_targets + a.target];
     const float scale = a.scales[slot];  // (read here: its latency overlaps the unit's loads)

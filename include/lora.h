@@ -66,7 +66,10 @@ enum {
                                   [-1, n_slots) or a malformed segment        */
     LORA_ERR_TIMEOUT = 8,      /* sticky device status: a bounded wait inside
                                   a kernel gave up                            */
-    LORA_ERR_WORKSPACE = 9     /* workspace smaller than lora_workspace_bytes */
+    LORA_ERR_WORKSPACE = 9,    /* workspace smaller than lora_workspace_bytes */
+    LORA_ERR_BOUNDS = 10       /* sticky device status, LORA_DEBUG builds only: an
+                                  index or page outside its buffer was about to be
+                                  used (the access was skipped or redirected) */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */

@@ -52,9 +52,23 @@ def test_header_compiles_as_plain_c(tmp_path):
                    check=True)
 
 
+def test_debug_library_exports_every_declared_symbol():
+    # the LORA_DEBUG build (bounds checks in the kernels) has the same boundary
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_lora_build", os.path.join(ROOT, "adapter_deltas_b200", "_build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    lib = b.build(debug=True)  # (no-op when it is current)
+    out = subprocess.run(["nm", "-D", "--defined-only", lib], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r" T (lora_\w+)$", out.stdout, flags=re.M))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+
+
 def test_status_strings(L):
     assert L.lora_status_string(0) == "LORA_OK"
     assert L.lora_status_string(L.LORA_ERR_WORKSPACE) == "LORA_ERR_WORKSPACE"
+    assert L.lora_status_string(L.LORA_ERR_BOUNDS) == "LORA_ERR_BOUNDS"
     assert L.lora_status_string(999) == "LORA_ERR_UNKNOWN"
 
 
