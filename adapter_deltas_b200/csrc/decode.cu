@@ -96,6 +96,7 @@ struct DecodeArgs {
   const float *scales;
   // plan path
   const int32_t *hdr;
+  int early;  // plan path (not expand-only, T <= kCachePerm): see early_prefetch
   const int32_t *perm;
   const int4 *items;
   int items_hdr;  // header word holding the item count to process
@@ -574,7 +575,7 @@ struct DecSmem {
   uint64_t *full, *empty; // [kMaxStages] each
   uint8_t *zero;          // 32 zero bytes: the expand's operand rows beyond the rank
   float *v;               // [kItemRows][r_max]: V of the current unit
-  int *misc;              // [0]: abort flag
+  int *misc;              // [0]: abort flag; [2]: early_prefetch's decision
   int4 *c_item;           // [kCacheItems]: slot, first grouped position, rows
   int4 *c_slot;           // [kCacheItems]: rank, A page, B^T page, scale bits (first target)
   int *c_perm;            // [kCachePerm]: row of each grouped position
@@ -841,6 +842,9 @@ struct UnitGeo {
   }
 };
 
+// When a CTA of a launch that may prefetch early (DecodeArgs::early) last
+// found no unit (%globaltimer, ns; one word per device, read by early_prefetch).
+__device__ unsigned long long g_idle_ns;
 __device__ __forceinline__ bool aborted(const DecSmem &S) { return *(volatile int *)S.misc != 0; }
 __device__ __forceinline__ void set_abort(const DecSmem &S) { *(volatile int *)S.misc = 1; }
 
@@ -915,6 +919,8 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
   };
   const int n_uneven = MODE == kFused ? uneven_ranges(a, S, n_items, U.nnu, U.nnt, lane) : 0;
   const int n_units = n_uneven > 0 ? n_uneven : U.total;
+  if (a.early && (int)blockIdx.x >= n_units && lane == 0)
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(&g_idle_ns), "l"(global_ns()) : "memory");
   int item = blockIdx.x / (NT * U.nnu), rem = blockIdx.x - item * (NT * U.nnu);
   const int step_item = gridDim.x / (NT * U.nnu), step_rem = gridDim.x - step_item * (NT * U.nnu);
   for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
@@ -1034,6 +1040,120 @@ __device__ void produce(const DecodeArgs &a, const DecSmem &S, int n_items, int 
     S.hdr[stage] = StageHdr{kUnitEnd, 0, 0, 0};
     mbar_arrive_expect_tx(&S.full[stage], 0);
   }
+}
+
+// ------------------------------------------------------------ early prefetch
+// Physical page of a slot's block as block_page() finds it, read from L2
+// only (no line of the page table is left in L1 for later reads).
+__device__ __forceinline__ int block_page_l2(const PoolView &p, int slot, long long first, long long bytes) {
+  if (p.log2_page < 0) return __ldcg(p.pt + (long long)slot * p.pps);
+  const long long pf = first >> p.log2_page, pl = (first + bytes - 1) >> p.log2_page;
+  return pf == pl ? __ldcg(p.pt + (long long)slot * p.pps + pf) : -1;
+}
+
+// A launch on a plan may start before the kernel ahead of it on the stream
+// has finished (programmatic dependent launch).  When that kernel is another
+// such decode launch, the CTAs that start first are those that took an SM
+// one of its CTAs without a unit gave back at once, and they would wait for
+// it to finish anyway; so they bring the units' tiles and activation rows
+// into L2 meanwhile: the first gridDim - n_units CTAs share the units (CTA
+// b: units b, b + n_early, ...).  A CTA without a unit stamps g_idle_ns; a
+// starting CTA counts itself early only if the stamp is under kEarlyNs old,
+// so a launch that starts behind any other kernel (a base GEMM), or alone,
+// skips all of this after one load.  The early CTAs read the plan and the
+// pool's tables as they stand (L2-only loads, so nothing stale stays in L1),
+// clamp every index into its buffer and use what they read for prefetch
+// addresses only: a plan that is being rewritten, or a stamp left by a launch
+// on another stream, costs a useless prefetch, never a wrong result.  All
+// threads load, the copy warp prefetches.
+constexpr unsigned long long kEarlyNs = 4000;
+template <int MODE>
+__device__ void early_prefetch(const DecodeArgs &a, const DecSmem &S, int tid) {
+  const int lane = tid & 31, warp = tid >> 5, T = a.T;
+  const PoolView &p = a.pool;
+  if (tid == 0) {
+    unsigned long long t;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(t) : "l"(&g_idle_ns) : "memory");
+    S.misc[2] = global_ns() - t < kEarlyNs;
+  }
+  __syncthreads();
+  if (!S.misc[2]) return;
+  const int n_ci = min(a.items_cap, kCacheItems);
+  if (tid < n_ci) {
+    const int4 d = __ldcg(a.items + tid);
+    const int slot = min(max(d.x, 0), p.n_slots - 1), first = min(max(d.y, 0), T);
+    S.c_item[tid] = make_int4(slot, first, min(max(d.z, 0), min(kItemRows, T - first)), 0);
+  }
+  for (int q = tid; q < T; q += kDecThreads) S.c_perm[q] = min(max(__ldcg(a.perm + q), 0), T - 1);
+  __syncthreads();
+  if (warp == kProdWarp) {
+    int n_items = lane == 0 ? __ldcg(a.hdr + a.items_hdr) : 0;
+    n_items = min(max(__shfl_sync(0xffffffffu, n_items, 0), 0), n_ci);
+    const UnitGeo<MODE> U(a, n_items);
+    const int NT = a.n_tgt;
+    const int n_uneven = MODE == kFused ? uneven_ranges(a, S, n_items, U.nnu, U.nnt, lane) : 0;
+    const int n_units = n_uneven > 0 ? n_uneven : U.total;
+    const int n_early = (int)gridDim.x - n_units;
+    const int nvi = a.d_in / 8, nvo = a.d_out / 8;
+    const long long tile_stride = (long long)a.r_max * a.kcv * 16;
+    for (int u0 = blockIdx.x; u0 < n_units && (int)blockIdx.x < n_early; u0 += 32 * n_early) {
+      // lane j: where unit u0 + j * n_early lies and its slot's record
+      const int u = u0 + lane * n_early;
+      int it = 0, ti = 0, e0 = 0, e1 = 0, r = 0, pa = -1, pb = -1;
+      if (u < n_units) {
+        if (n_uneven > 0) {
+          int lo_t = 0, hi_t = n_items - 1;
+          while (lo_t < hi_t) {
+            const int mid = (lo_t + hi_t + 1) >> 1;
+            if (NT * S.c_pref[mid] <= u) lo_t = mid;
+            else hi_t = mid - 1;
+          }
+          it = lo_t;
+          const int k = S.c_pref[lo_t + 1] - S.c_pref[lo_t];
+          const int local = u - NT * S.c_pref[lo_t];
+          ti = local / k;
+          const int j = local - ti * k;
+          e0 = j * U.nnt / k;
+          e1 = (j + 1) * U.nnt / k;
+        } else {
+          it = u / (NT * U.nnu);
+          const int rem = u - it * (NT * U.nnu);
+          ti = rem / U.nnu;
+          e0 = (rem - ti * U.nnu) * U.npu;
+          e1 = MODE == kShrinkOnly ? e0 : min(e0 + U.npu, U.nnt);
+        }
+        const int slot = S.c_item[it].x;
+        r = min(max(__ldcg(p.rank + (long long)slot * p.n_targets + a.tgt[ti]), 0), a.r_max);
+        pa = block_page_l2(p, slot, a.a_off[ti], (long long)a.r_max * a.d_in * 2);
+        pb = block_page_l2(p, slot, a.bt_off[ti], (long long)a.r_max * a.d_out * 2);
+      }
+      const int nu = min(32, (n_units - u0 + n_early - 1) / n_early);
+      for (int j = 0; j < nu; ++j) {
+        const int uit = __shfl_sync(0xffffffffu, it, j), uti = __shfl_sync(0xffffffffu, ti, j);
+        const int ue0 = __shfl_sync(0xffffffffu, e0, j), ue1 = __shfl_sync(0xffffffffu, e1, j);
+        const int ur = __shfl_sync(0xffffffffu, r, j);
+        const int upa = __shfl_sync(0xffffffffu, pa, j), upb = __shfl_sync(0xffffffffu, pb, j);
+        const int4 d = S.c_item[uit];
+        if (ur == 0 || d.z == 0) continue;
+        for (int q = lane; q < U.nkt + (ue1 - ue0); q += 32) {  // adapter rows, one tile per lane
+          const bool sq = q < U.nkt;
+          const int tq = sq ? q : ue0 + (q - U.nkt);
+          const int page = sq ? upa : upb;
+          const long long off = (sq ? a.a_off[uti] : a.bt_off[uti]) + tq * tile_stride;
+          if (page >= 0 && page < p.n_pages)
+            bulk_prefetch_l2(page_addr(p, page, off),
+                             (uint32_t)ur * (uint32_t)min(a.kcv, (sq ? nvi : nvo) - tq * a.kcv) * 16u);
+        }
+        if (lane < d.z) {  // the item's x rows and its y rows in the unit's columns
+          const int row = S.c_perm[d.y + lane];
+          bulk_prefetch_l2(a.x + (long long)(row / a.x_div) * a.ldx, (uint32_t)nvi * 16u);
+          const int v0 = ue0 * a.kcv, v1 = min(ue1 * a.kcv, nvo);
+          if (v1 > v0) bulk_prefetch_l2(a.y + (long long)row * a.ldy + a.y_col[uti] + (long long)v0 * 8, (uint32_t)(v1 - v0) * 16u);
+        }
+      }
+    }
+  }
+  __syncthreads();  // (the shared arrays are rewritten from the plan next)
 }
 
 // Consumer warps: the contractions, out of the ring.
@@ -1214,6 +1334,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_min_blocks(JB)) decode_kernel
     S.tg[2 * kMaxMulti + tid] = a.y_col[tid];
   }
   __syncthreads();
+  if (a.early && !a.stall) early_prefetch<MODE>(a, S, tid);
   griddep_wait();
   griddep_launch_dependents();
   const int n_items = a.ids ? fused_group(a, S, tid) : plan_cache(a, S, tid);  // every thread
@@ -1352,6 +1473,7 @@ int launch_decode(lora_pool *pool, const DecodeCall &c, cudaStream_t st) {
   a.ldy = c.ldy;
   a.scales = c.scales;
   const PlanLayout L = plan_layout(c.T);
+  a.early = !c.ids && c.mode != kExpandOnly && c.T <= kCachePerm;
   if (c.ids) {
     a.hdr = nullptr;
     a.perm = nullptr;
