@@ -26,7 +26,8 @@
  *    example torch tensor storage); the library never frees them.
  *  - stream is a cudaStream_t passed as void*; NULL is the legacy default
  *    stream.  Compute calls are asynchronous on that stream and never
- *    synchronise the host, never allocate, and may be captured in a CUDA graph.
+ *    synchronise the host or allocate; those that take a workspace may be
+ *    captured in a CUDA graph.
  *  - bf16 tensors are row-major with a leading dimension (ld*) counted in
  *    elements.  x, y, weights and workspace must be 16-byte aligned, and
  *    d_in, d_out, ldx and ldy must be multiples of 8, else LORA_ERR_ALIGNMENT.
